@@ -1,0 +1,535 @@
+#!/usr/bin/env python
+"""Throughput of the exact-attention kernels on B200, one JSON line per run.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--no-secondary] [--no-cpu-baseline]
+
+A step is one call of the library over one batch of the workload with inputs
+resident in device memory; K steps run back to back on rotating input sets whose
+total size exceeds twice the L2 cache, bracketed by a barrier and a device
+synchronisation, timed with CUDA events on the launching stream.  Under torchrun
+each rank runs its own replica (weak scaling) and the slowest rank's time counts.
+
+The headline workload is the batched ViT-B/16 attention layer (B=64, H=12, N=196,
+d=64, bf16 forward).  With secondary measurements on (the default at one GPU) the
+line also carries the long causal GQA prefill, the non-causal N=8192 prefill, the
+causal training step (forward + backward) and the paged decode step.
+
+`--impl reference` times the fp64 CPU oracle on a bounded sample of the same
+workload (the only other implementation of this method here).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "attention TFLOP/s & % of B200 BF16 tensor peak; paged-decode HBM GB/s"
+L2_BYTES = 126 * 2**20
+NOMINAL_BF16_TFLOPS = 2250.0
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return FALLBACK, "fallback"
+
+
+def kernel_sources_sha() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "exact_attention_128_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel: str):
+    """Per-launch DRAM bytes from a committed ncu summary, if taken on the current sources."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            t = json.load(f)
+    except (OSError, ValueError):
+        return None
+    e = t.get(kernel)
+    if not e or e.get("src_sha") != kernel_sources_sha():
+        return None
+    return e.get("bytes_per_launch")
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"fa_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.fh, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        self.t0 = time.time()
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        sm, mx, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- helpers
+def dist_setup():
+    import torch
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def n_rotations(bytes_per_set: int) -> int:
+    return max(2, math.ceil(2 * L2_BYTES / max(bytes_per_set, 1)) + 1)
+
+
+def timed_loop(fns, steps, warmup, world):
+    """Run fns[i % len(fns)]() for warmup then `steps` iterations; device-timed ms."""
+    import torch
+
+    for i in range(warmup):
+        fns[i % len(fns)]()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    st = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for i in range(steps):
+        fns[i % len(fns)]()
+    e1.record(st)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    return max_over_ranks(e0.elapsed_time(e1), world)
+
+
+# ----------------------------------------------------------------------------- workloads
+def dense_fwd_step_fns(case, dev, rot=None):
+    """Device-resident rotating input sets and one C-ABI fa_fwd call per step."""
+    import ctypes
+
+    import torch
+
+    import exact_attention_128_b200 as fa
+
+    q, k, v = case.make()
+    set_bytes = 2 * q.numel() * q.element_size() + k.numel() * k.element_size() * 2
+    rot = rot or n_rotations(set_bytes)
+    L = fa.lib()
+    sets, fns = [], []
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    for i in range(rot):
+        qq, kk, vv = (qd, kd, vd) if i == 0 else (qd.clone(), kd.clone(), vd.clone())
+        o = torch.empty_like(qq)
+        lse = torch.empty(case.B, case.Hq, case.Nq, device=dev, dtype=torch.float32)
+        sets.append((qq, kk, vv, o, lse))
+        args = [ctypes.c_void_p(t.data_ptr()) for t in (qq, kk, vv, o, lse)] + [
+            case.B, case.Hq, case.Hkv, case.Nq, case.Nkv, case.d, ctypes.c_float(case.scale), int(case.causal),
+            fa.FA_DTYPE_BF16, ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)]
+
+        def fn(args=args):
+            s = L.fa_fwd(*args)
+            if s != 0:
+                raise fa.FAError("fa_fwd", s)
+
+        fns.append(fn)
+    return fns, sets, (q, k, v), rot * set_bytes
+
+
+def e2e_fwd(case, dev, steps, warmup, world):
+    """Same metric through the public API with pinned host buffers: H2D q,k,v, fwd, D2H o,lse."""
+    import torch
+
+    import exact_attention_128_b200 as fa
+
+    q, k, v = (t.pin_memory() for t in case.make())
+    qd, kd, vd = torch.empty_like(q, device=dev), torch.empty_like(k, device=dev), torch.empty_like(v, device=dev)
+    oh = torch.empty_like(q).pin_memory()
+    lh = torch.empty(case.B, case.Hq, case.Nq, dtype=torch.float32).pin_memory()
+    od, ld = torch.empty_like(qd), torch.empty(case.B, case.Hq, case.Nq, device=dev, dtype=torch.float32)
+
+    def step():
+        qd.copy_(q, non_blocking=True)
+        kd.copy_(k, non_blocking=True)
+        vd.copy_(v, non_blocking=True)
+        fa.fwd(qd, kd, vd, causal=case.causal, scale=case.scale, out=od, lse=ld)
+        oh.copy_(od, non_blocking=True)
+        lh.copy_(ld, non_blocking=True)
+
+    ms = timed_loop([step], steps, warmup, world)
+    h2d = sum(t.numel() * t.element_size() for t in (q, k, v))
+    d2h = oh.numel() * oh.element_size() + lh.numel() * 4
+    return ms, h2d, d2h
+
+
+def measure_dense_fwd(case, dev, steps, warmup, world, peaks, peak_key="bf16_tflops"):
+    fns, sets, host, rot_bytes = dense_fwd_step_fns(case, dev)
+    ms = timed_loop(fns, steps, warmup, world)
+    flops = case.fwd_flops()
+    per_step_ms = ms / steps
+    tflops = flops / (per_step_ms * 1e-3) / 1e12
+    kname = f"fa_fwd_bf16_kernel<{case.d},{str(case.causal).lower()}>"
+    peak = peaks[peak_key]
+    roof = {"bound": "tensor", "achieved": round(tflops, 2), "peak": peak, "unit": "TFLOP/s",
+            "frac": round(tflops / peak, 4), "traffic": traffic_for(kname), "kernel": kname,
+            "peak_kind": peak_key, "frac_of_nominal_2250": round(tflops / NOMINAL_BF16_TFLOPS, 4),
+            "algorithmic_flops_per_launch": flops}
+    return {"ms": ms, "per_step_ms": per_step_ms, "tflops": tflops, "roofline": roof, "rot_bytes": rot_bytes,
+            "launches_per_step": 1}
+
+
+def measure_train(case, dev, steps, warmup, world, peaks):
+    """Forward + backward (recompute) per step."""
+    import torch
+
+    import exact_attention_128_b200 as fa
+
+    q, k, v, do = case.make(with_grad_output=True)
+    set_bytes = sum(t.numel() * t.element_size() for t in (q, k, v, do)) * 2
+    rot = n_rotations(set_bytes)
+    qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
+    sets = []
+    ws = torch.empty(fa.bwd_workspace_size(case.B, case.Hq, case.Nq, case.d), device=dev, dtype=torch.uint8)
+    for i in range(rot):
+        s = (qd, kd, vd, dod) if i == 0 else tuple(t.clone() for t in (qd, kd, vd, dod))
+        sets.append(s)
+
+    def mk(s):
+        def step():
+            o, lse = fa.fwd(s[0], s[1], s[2], causal=case.causal, scale=case.scale)
+            fa.bwd(s[0], s[1], s[2], o, lse, s[3], causal=case.causal, scale=case.scale, workspace=ws)
+        return step
+
+    fns = [mk(s) for s in sets]
+    ms = timed_loop(fns, steps, warmup, world)
+    fwd = case.fwd_flops()
+    flops = fwd * 3.5  # forward 2 contractions + backward 5 (score recompute included)
+    per = ms / steps
+    tflops = flops / (per * 1e-3) / 1e12
+    peak = peaks["bf16_tflops"]
+    return {"per_step_ms": per, "tflops": tflops,
+            "roofline": {"bound": "tensor", "achieved": round(tflops, 2), "peak": peak, "unit": "TFLOP/s",
+                         "frac": round(tflops / peak, 4), "frac_of_nominal_2250": round(tflops / NOMINAL_BF16_TFLOPS, 4),
+                         "algorithmic_flops_per_step": flops}}
+
+
+def measure_decode(pc, dev, steps, warmup, world, peaks):
+    import ctypes
+
+    import torch
+
+    import exact_attention_128_b200 as fa
+    from exact_attention_128_b200.workloads import PagedCase
+
+    inp = pc.make()
+    kvb = PagedCase.kv_bytes(inp["ctx_lens"].tolist(), pc.Hkv, pc.d)
+    set_bytes = inp["k_cache"].numel() * 4
+    rot = n_rotations(set_bytes)
+    L = fa.lib()
+    base = {n: inp[n].to(dev) for n in ("q", "k_cache", "v_cache", "block_table", "ctx_lens")}
+    need = fa.paged_decode_workspace_size(pc.R, pc.Hq, pc.d, pc.max_blocks_per_seq, pc.block_size)
+    fns, keep = [], []
+    for i in range(rot):
+        s = base if i == 0 else {n: t.clone() for n, t in base.items()}
+        o = torch.empty_like(s["q"])
+        lse = torch.empty(pc.R, pc.Hq, device=dev, dtype=torch.float32)
+        ws = torch.empty(need, device=dev, dtype=torch.uint8)
+        keep.append((s, o, lse, ws))
+        args = [ctypes.c_void_p(s[n].data_ptr()) for n in ("q", "k_cache", "v_cache", "block_table", "ctx_lens")]
+        args += [ctypes.c_void_p(o.data_ptr()), ctypes.c_void_p(lse.data_ptr()), pc.R, pc.Hq, pc.Hkv, pc.d,
+                 pc.block_size, pc.max_blocks_per_seq, inp["num_blocks"], ctypes.c_float(pc.scale),
+                 fa.FA_DTYPE_BF16, ctypes.c_void_p(ws.data_ptr()), need,
+                 ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)]
+
+        def fn(args=args):
+            st = L.fa_paged_decode(*args)
+            if st != 0:
+                raise fa.FAError("fa_paged_decode", st)
+
+        fns.append(fn)
+    ms = timed_loop(fns, steps, warmup, world)
+    per = ms / steps
+    gbs = kvb / (per * 1e-3) / 1e9
+    peak = peaks["hbm_gbs"]
+    return {"per_step_ms": per, "gbs": gbs, "kv_bytes": kvb,
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(gbs / peak, 4), "frac_of_nominal_8000": round(gbs / NOMINAL_HBM_GBS, 4),
+                         "algorithmic_bytes_per_step": kvb, "kernels": ["fa_paged_decode_kernel",
+                                                                        "fa_paged_decode_combine_kernel"]}}
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def cpu_oracle_dense(case, budget_s=12.0):
+    """Time the fp64 oracle on whole heads of the workload until ~budget_s of CPU work."""
+    import numpy as np
+
+    from oracle import attention_fp64 as ora
+
+    q, k, v = case.make()
+    qn, kn, vn = (ora.to_f64(t) for t in (q, k, v))
+    G = case.Hq // case.Hkv
+    heads = [(b, h) for b in range(case.B) for h in range(case.Hq)]
+    done, t0 = 0, time.perf_counter()
+    while time.perf_counter() - t0 < budget_s:
+        b, h = heads[done % len(heads)]
+        ora.attention_head(qn[b, h], kn[b, h // G], vn[b, h // G], case.scale, case.causal)
+        done += 1
+    dt = time.perf_counter() - t0
+    flops = case.fwd_flops() / len(heads) * done
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": oracle_threads(), "kind": "oracle",
+            "sample": f"{done} whole (b,h) heads of {case.name} ({done / len(heads):.2f} passes), "
+                      f"{dt:.1f} s, NumPy fp64 materialising the score matrix"}
+
+
+def reference_line(case, args):
+    """The oracle as the reference arm: W + K steps, each step whole heads of the workload.
+
+    Heads per step are sized from one probe head so the whole run stays within ~90 s.
+    """
+    from oracle import attention_fp64 as ora
+
+    q, k, v = case.make()
+    qn, kn, vn = (ora.to_f64(t) for t in (q, k, v))
+    G = case.Hq // case.Hkv
+    heads = [(b, h) for b in range(case.B) for h in range(case.Hq)]
+    t0 = time.perf_counter()
+    ora.attention_head(qn[0, 0], kn[0, 0], vn[0, 0], case.scale, case.causal)
+    t_head = max(time.perf_counter() - t0, 1e-4)
+    per_step = max(1, min(len(heads), int(90.0 / ((args.steps + args.warmup) * t_head))))
+    idx = 0
+
+    def step():
+        nonlocal idx
+        for _ in range(per_step):
+            b, h = heads[idx % len(heads)]
+            idx += 1
+            ora.attention_head(qn[b, h], kn[b, h // G], vn[b, h // G], case.scale, case.causal)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    flops = case.fwd_flops() / len(heads) * per_step * args.steps
+    value = flops / dt / 1e12
+    cb = {"value": value, "unit": "TFLOP/s", "cores": oracle_threads(), "kind": "oracle",
+          "sample": f"{per_step} whole (b,h) head(s) of {case.name} per step, {args.steps} steps, {dt:.1f} s"}
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": case.name, "B": case.B, "Hq": case.Hq, "Hkv": case.Hkv, "N": case.Nq,
+                       "d": case.d, "causal": case.causal, "sample_heads_per_step": per_step},
+            "cpu_baseline": cb,
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+# ----------------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="vit_b16_batched_fwd_bf16")
+    ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    from exact_attention_128_b200 import workloads as W
+
+    dense = {c.name: c for c in [W.VIT_BATCHED_BF16, W.GQA_PREFILL_CAUSAL, *W.prefill_sweep()]}
+    if args.workload not in dense:
+        ap.error(f"unknown workload {args.workload}; choose from {sorted(dense)}")
+    case = dense[args.workload]
+    peaks, peaks_kind = load_peaks()
+
+    if args.impl == "reference":
+        if int(os.environ.get("RANK", "0")) != 0:
+            return  # rank 0 alone times the CPU oracle
+        print(json.dumps(reference_line(case, args)))
+        return
+
+    import torch
+
+    import exact_attention_128_b200 as fa
+
+    world, rank, local = dist_setup()
+    dev = torch.device("cuda", local)
+    fa.lib()
+    fa.device_status(reset=True)
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    head = measure_dense_fwd(case, dev, args.steps, args.warmup, world, peaks)
+    clocks = sampler.stop()
+
+    e2e = None
+    if not args.no_e2e:
+        e_steps = max(3, min(args.steps, 200))
+        ms, h2d, d2h = e2e_fwd(case, dev, e_steps, args.warmup, world)
+        e2e = {"value": round(world * case.fwd_flops() * e_steps / (ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e_steps,
+               "ms_per_step": round(ms / e_steps, 4)}
+
+    secondary = {}
+    if not args.no_secondary and world == 1:
+        for c in (W.GQA_PREFILL_CAUSAL, W.prefill_sweep()[3]):
+            if c.name == case.name:
+                continue
+            r = measure_dense_fwd(c, dev, max(20, args.steps // 50), 5, world, peaks)
+            secondary[c.name] = {"value": round(r["tflops"], 2), "unit": "TFLOP/s",
+                                 "ms_per_step": round(r["per_step_ms"], 4), "roofline": r["roofline"]}
+            torch.cuda.empty_cache()
+        try:
+            r = measure_train(W.TRAIN_CAUSAL, dev, max(10, args.steps // 100), 3, world, peaks)
+            secondary[W.TRAIN_CAUSAL.name] = {"value": round(r["tflops"], 2), "unit": "TFLOP/s",
+                                              "ms_per_step": round(r["per_step_ms"], 4), "roofline": r["roofline"]}
+        except fa.FAError as e:
+            secondary[W.TRAIN_CAUSAL.name] = {"unavailable": str(e)}
+        torch.cuda.empty_cache()
+        r = measure_decode(W.PAGED_DECODE, dev, max(50, args.steps // 4), 10, world, peaks)
+        secondary[W.PAGED_DECODE.name] = {"value": round(r["gbs"], 1), "unit": "GB/s",
+                                          "ms_per_step": round(r["per_step_ms"], 5), "roofline": r["roofline"]}
+
+    status = fa.device_status(reset=True)
+    if status != 0:
+        raise SystemExit(f"device status {status} after the run")
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_oracle_dense(case, budget_s=12.0)
+
+    value = world * case.fwd_flops() * args.steps / (head["ms"] * 1e-3) / 1e12
+    line = {
+        "metric": METRIC,
+        "value": round(value, 3),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(head["per_step_ms"], 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": case.name, "B": case.B, "Hq": case.Hq, "Hkv": case.Hkv, "N": case.Nq, "d": case.d,
+                   "causal": case.causal, "parallelism": f"replicas{world}",
+                   "l2": f"rotating input sets, {head['rot_bytes'] / 2**20:.0f} MiB > 2x L2"},
+        "roofline": head["roofline"],
+        "peaks": peaks_kind,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": head["launches_per_step"] * args.steps,
+        "clocks": clocks,
+        "secondary": secondary,
+    }
+    if rank == 0:
+        print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

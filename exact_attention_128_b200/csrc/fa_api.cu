@@ -1,0 +1,224 @@
+// fa_api.cu — the C ABI (include/fa.h): argument validation, TMA descriptor
+// encoding and kernel launches.  Everything that computes runs in the kernels;
+// this file only checks arguments and launches them on the caller's stream.
+#include <cmath>
+#include <cstdio>
+#include <mutex>
+
+#include "common.cuh"
+#include "decode.cuh"
+#include "fwd_bf16.cuh"
+#include "fwd_f32.cuh"
+#include "bwd_bf16.cuh"
+
+namespace {
+
+using namespace fa;
+
+uint64_t g_wait_ns = 200000000ull;  // 200 ms per wait
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 3-D bf16 map over [z][y][x] = [planes][rows][d] with a (64, box_rows, 1) box and the
+// 128-byte swizzle; rows past `rows` read as zeros.
+bool make_map_bf16(CUtensorMap* m, const void* base, int d, int rows, int planes, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(rows), cuuint64_t(planes)};
+  cuuint64_t strides[2] = {cuuint64_t(d) * 2, cuuint64_t(d) * 2 * cuuint64_t(rows)};
+  cuuint32_t box[3] = {64, cuuint32_t(box_rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename K>
+cudaError_t set_smem(K kernel, int bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+fa_status launched() { return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA; }
+
+template <int D, bool CAUSAL>
+fa_status launch_fwd_bf16(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                          const FwdBf16Params& prm, int B, int Hq, int Nq, cudaStream_t st) {
+  using C = FwdCfg<D>;
+  auto kern = fa_fwd_bf16_kernel<D, CAUSAL>;
+  if (set_smem(kern, C::SMEM) != cudaSuccess) return FA_ERR_CUDA;
+  dim3 grid((Nq + 2 * C::BM - 1) / (2 * C::BM), B * Hq);
+  kern<<<grid, C::THREADS, C::SMEM, st>>>(mq, mk, mv, prm);
+  return launched();
+}
+
+__global__ void selftest_wait_kernel(uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+    mbar_wait(&bar, 0, limit_ns, &abort_flag, 900);  // nothing arrives: must run out
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* fa_status_string(fa_status s) {
+  switch (s) {
+    case FA_OK: return "ok";
+    case FA_ERR_INVALID_ARG: return "invalid argument";
+    case FA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case FA_ERR_CUDA: return "CUDA error";
+    case FA_ERR_WORKSPACE: return "workspace missing or too small";
+    case FA_ERR_DEVICE_TIMEOUT: return "bounded in-kernel wait timed out";
+  }
+  return "unknown status";
+}
+
+int fa_version(void) { return 10000; }
+
+void fa_set_wait_limit_ns(uint64_t ns) { g_wait_ns = ns < 1000 ? 1000 : ns; }
+
+fa_status fa_device_status(int reset) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return FA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, fa::g_status, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
+  if (reset) {
+    int z = 0;
+    if (cudaMemcpyToSymbol(fa::g_status, &z, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
+    if (cudaMemcpyToSymbol(fa::g_status_where, &z, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
+  }
+  return static_cast<fa_status>(v);
+}
+
+fa_status fa_selftest_wait_timeout(void* stream) {
+  selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(g_wait_ns);
+  return launched();
+}
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Nq,
+                 int Nkv, int d, float scale, int causal, fa_dtype dtype, void* stream) {
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq <= 0 || Nkv <= 0 || d <= 0) return FA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  if (causal && Nq > Nkv) return FA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
+    return FA_ERR_INVALID_ARG;
+  if (long(B) * Hq > 65535) return FA_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  if (dtype == FA_DTYPE_F32) {
+    if (d != 64) return FA_ERR_UNSUPPORTED;
+    FwdF32Params prm{static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
+                     static_cast<float*>(o), lse, Hq, Hkv, Nq, Nkv, scale, causal};
+    dim3 grid((Nq + f32::BQ - 1) / f32::BQ, B * Hq);
+    fa_fwd_f32_kernel<<<grid, f32::THREADS, 0, st>>>(prm);
+    return launched();
+  }
+  if (dtype != FA_DTYPE_BF16) return FA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+
+  CUtensorMap mq, mk, mv;
+  if (!make_map_bf16(&mq, q, d, Nq, B * Hq, 128) || !make_map_bf16(&mk, k, d, Nkv, B * Hkv, 128) ||
+      !make_map_bf16(&mv, v, d, Nkv, B * Hkv, 128))
+    return FA_ERR_CUDA;
+  FwdBf16Params prm{static_cast<__nv_bfloat16*>(o), lse, Hq, Hkv, Nq, Nkv,
+                    scale * 1.4426950408889634f, g_wait_ns};
+  if (d == 64)
+    return causal ? launch_fwd_bf16<64, true>(mq, mk, mv, prm, B, Hq, Nq, st)
+                  : launch_fwd_bf16<64, false>(mq, mk, mv, prm, B, Hq, Nq, st);
+  return causal ? launch_fwd_bf16<128, true>(mq, mk, mv, prm, B, Hq, Nq, st)
+                : launch_fwd_bf16<128, false>(mq, mk, mv, prm, B, Hq, Nq, st);
+}
+
+size_t fa_bwd_workspace_size(int B, int Hq, int Nq, int d) {
+  if (B <= 0 || Hq <= 0 || Nq <= 0 || d <= 0) return 0;
+  const size_t rows = size_t(B) * Hq * Nq;
+  return align256(rows * d * sizeof(float)) + align256(rows * sizeof(float));
+}
+
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+                 void* dq, void* dk, void* dv, fa_dtype grad_dtype, int B, int Hq, int Hkv, int Nq, int Nkv, int d,
+                 float scale, int causal, fa_dtype dtype, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq <= 0 || Nkv <= 0 || d <= 0) return FA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  if (causal && Nq > Nkv) return FA_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, o, dO, dq, dk, dv};
+  for (const void* ptr : ptrs)
+    if (!aligned(ptr, 16)) return FA_ERR_INVALID_ARG;
+  if (!aligned(lse, 4)) return FA_ERR_INVALID_ARG;
+  if (dtype != FA_DTYPE_BF16) return FA_ERR_UNSUPPORTED;
+  if (grad_dtype != FA_DTYPE_F32 && grad_dtype != FA_DTYPE_BF16) return FA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (long(B) * Hq > 65535) return FA_ERR_UNSUPPORTED;
+  const size_t need = fa_bwd_workspace_size(B, Hq, Nq, d);
+  if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return FA_ERR_WORKSPACE;
+  return fa::bwd_launch(q, k, v, o, lse, dO, dq, dk, dv, grad_dtype, B, Hq, Hkv, Nq, Nkv, d, scale, causal,
+                        workspace, static_cast<cudaStream_t>(stream), g_wait_ns);
+}
+
+size_t fa_paged_decode_workspace_size(int R, int Hq, int d, int max_blocks_per_seq, int block_size) {
+  if (R <= 0 || Hq <= 0 || d <= 0 || max_blocks_per_seq <= 0 || block_size <= 0) return 0;
+  const size_t splits = size_t((max_blocks_per_seq + dec::CHUNK - 1) / dec::CHUNK);
+  return align256(size_t(R) * Hq * splits * d * sizeof(float)) + align256(size_t(R) * Hq * splits * sizeof(float));
+}
+
+fa_status fa_paged_decode(const void* q, const void* k_cache, const void* v_cache, const int* block_table,
+                          const int* ctx_lens, void* o, float* lse, int R, int Hq, int Hkv, int d, int block_size,
+                          int max_blocks_per_seq, int num_blocks, float scale, fa_dtype dtype, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+  if (!q || !k_cache || !v_cache || !block_table || !ctx_lens || !o) return FA_ERR_INVALID_ARG;
+  if (R <= 0 || Hq <= 0 || Hkv <= 0 || d <= 0 || block_size <= 0 || max_blocks_per_seq <= 0 || num_blocks <= 0)
+    return FA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(o, 16) ||
+      !aligned(block_table, 4) || !aligned(ctx_lens, 4) || (lse && !aligned(lse, 4)))
+    return FA_ERR_INVALID_ARG;
+  if (dtype != FA_DTYPE_BF16 || d != dec::D || block_size != dec::BS) return FA_ERR_UNSUPPORTED;
+  if (Hq / Hkv > dec::MAX_G || R > 65535 || Hkv > 65535) return FA_ERR_UNSUPPORTED;
+  const size_t need = fa_paged_decode_workspace_size(R, Hq, d, max_blocks_per_seq, block_size);
+  if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return FA_ERR_WORKSPACE;
+  const int max_splits = (max_blocks_per_seq + dec::CHUNK - 1) / dec::CHUNK;
+  float* part_o = static_cast<float*>(workspace);
+  float* part_lse =
+      reinterpret_cast<float*>(static_cast<char*>(workspace) + align256(size_t(R) * Hq * max_splits * d * 4));
+  DecodeParams prm{static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k_cache),
+                   static_cast<const __nv_bfloat16*>(v_cache), block_table, ctx_lens,
+                   static_cast<__nv_bfloat16*>(o), lse, part_o, part_lse, R, Hq, Hkv, max_blocks_per_seq,
+                   num_blocks, max_splits, scale * 1.4426950408889634f};
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (set_smem(fa_paged_decode_kernel, dec::SMEM) != cudaSuccess) return FA_ERR_CUDA;
+  fa_paged_decode_kernel<<<dim3(max_splits, Hkv, R), dec::WARPS * 32, dec::SMEM, st>>>(prm);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  fa_paged_decode_combine_kernel<<<R * Hq, dec::D, 0, st>>>(prm);
+  return launched();
+}
+
+}  // extern "C"

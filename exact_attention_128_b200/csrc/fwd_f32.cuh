@@ -1,0 +1,158 @@
+// fwd_f32.cuh — fp32 forward pass on the CUDA cores (head dim 64).
+//
+// Exact attention, softmax(Q K^T * scale) V ("Autoatención, kernels CUDA y
+// FlashAttention" §1), evaluated tile by tile with the online-softmax recurrence of
+// "FlashAttention" (paweldubiel.com notes), "No basta con promediar los resultados de
+// los bloques": running maximum m, sum l and numerator u; when a tile raises the
+// maximum, l and u are multiplied by e^{m - m'} before the tile's terms are added.
+//
+// fp32 inputs need fp32 products (TF32 tensor-core inputs would lose ~3 decimal
+// digits), so this kernel uses FFMA.  It serves the small fp32 ViT layer; the bf16
+// tensor-core kernel is the throughput path.
+#pragma once
+#include "common.cuh"
+
+namespace fa {
+
+namespace f32 {
+constexpr int D = 64;
+constexpr int BQ = 64;        // query rows per CTA
+constexpr int BK = 32;        // keys per tile
+constexpr int THREADS = 256;  // 4 threads per query row
+constexpr int KPAD = D + 1;   // padded K row (bank-conflict free score loop)
+constexpr int PPAD = BK + 1;  // padded P row
+}  // namespace f32
+
+struct FwdF32Params {
+  const float* q;
+  const float* k;
+  const float* v;
+  float* o;
+  float* lse;
+  int Hq, Hkv, Nq, Nkv;
+  float scale;
+  int causal;
+};
+
+__global__ void __launch_bounds__(f32::THREADS) fa_fwd_f32_kernel(const FwdF32Params p) {
+  using namespace f32;
+  __shared__ float Ks[BK * KPAD];
+  __shared__ __align__(16) float Vs[BK * D];
+  __shared__ float Ps[BQ * PPAD];
+
+  const int tid = threadIdx.x;
+  const int r = tid >> 2;   // query row within the tile
+  const int qd = tid & 3;   // quarter: keys qd, qd+4, ... of a tile; output columns [16*qd, 16*qd+16)
+  const int bh = blockIdx.y;
+  const int b = bh / p.Hq, h = bh % p.Hq;
+  const int hk = h / (p.Hq / p.Hkv);
+  const int q0 = blockIdx.x * BQ;
+  const int row = q0 + r;
+  const bool row_ok = row < p.Nq;
+  const int off = p.Nkv - p.Nq;  // bottom-right causal alignment
+
+  const float* Qh = p.q + (size_t(bh) * p.Nq) * D;
+  const float* Kh = p.k + (size_t(b) * p.Hkv + hk) * size_t(p.Nkv) * D;
+  const float* Vh = p.v + (size_t(b) * p.Hkv + hk) * size_t(p.Nkv) * D;
+
+  float qr[D];
+#pragma unroll
+  for (int c = 0; c < D; c += 4) {
+    float4 t = row_ok ? *reinterpret_cast<const float4*>(Qh + size_t(row) * D + c) : make_float4(0, 0, 0, 0);
+    qr[c] = t.x; qr[c + 1] = t.y; qr[c + 2] = t.z; qr[c + 3] = t.w;
+  }
+
+  float m = -INFINITY, l = 0.f;
+  float acc[16];
+#pragma unroll
+  for (int c = 0; c < 16; ++c) acc[c] = 0.f;
+
+  // keys visible to this CTA's last row
+  int kv_end = p.Nkv;
+  if (p.causal) kv_end = min(p.Nkv, min(q0 + BQ, p.Nq) - 1 + off + 1);
+  const int ntiles = (kv_end + BK - 1) / BK;
+  // per-row limit on visible keys
+  const int row_limit = p.causal ? min(p.Nkv, row + off + 1) : p.Nkv;
+
+  for (int t = 0; t < ntiles; ++t) {
+    const int k0 = t * BK;
+    // stage K (padded rows) and V tiles; rows past Nkv are zero
+    for (int i = tid; i < BK * (D / 4); i += THREADS) {
+      const int kr = i / (D / 4), c4 = (i % (D / 4)) * 4;
+      float4 kk = make_float4(0, 0, 0, 0), vv = make_float4(0, 0, 0, 0);
+      if (k0 + kr < p.Nkv) {
+        kk = *reinterpret_cast<const float4*>(Kh + size_t(k0 + kr) * D + c4);
+        vv = *reinterpret_cast<const float4*>(Vh + size_t(k0 + kr) * D + c4);
+      }
+      float* kd = Ks + kr * KPAD + c4;
+      kd[0] = kk.x; kd[1] = kk.y; kd[2] = kk.z; kd[3] = kk.w;
+      *reinterpret_cast<float4*>(Vs + kr * D + c4) = vv;
+    }
+    __syncthreads();
+
+    constexpr int KQ = BK / 4;  // keys per thread
+    float s[KQ];
+#pragma unroll
+    for (int c = 0; c < KQ; ++c) s[c] = 0.f;
+#pragma unroll
+    for (int dd = 0; dd < D; ++dd) {
+      const float qv = qr[dd];
+#pragma unroll
+      for (int c = 0; c < KQ; ++c) s[c] = fmaf(qv, Ks[(c * 4 + qd) * KPAD + dd], s[c]);
+    }
+    float mx = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < KQ; ++c) {
+      const int key = k0 + c * 4 + qd;
+      s[c] = (key < row_limit) ? s[c] * p.scale : -INFINITY;
+      mx = fmaxf(mx, s[c]);
+    }
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    const float m_new = fmaxf(m, mx);
+    // a row whose visible keys all lie in later tiles keeps m = -inf; use 0 as the base
+    const float base = (m_new == -INFINITY) ? 0.f : m_new;
+    const float alpha = expf(m - base);  // e^{m - m'}; 0 when m = -inf
+    float rs = 0.f;
+#pragma unroll
+    for (int c = 0; c < KQ; ++c) {
+      const float e = expf(s[c] - base);
+      rs += e;
+      Ps[r * PPAD + c * 4 + qd] = e;
+    }
+    rs += __shfl_xor_sync(0xffffffffu, rs, 1);
+    rs += __shfl_xor_sync(0xffffffffu, rs, 2);
+    l = l * alpha + rs;
+    m = m_new;
+#pragma unroll
+    for (int c = 0; c < 16; ++c) acc[c] *= alpha;
+    __syncthreads();
+
+    const int kn = min(BK, kv_end - k0);
+    for (int kk = 0; kk < kn; ++kk) {
+      const float pv = Ps[r * PPAD + kk];
+      const float4* vrow = reinterpret_cast<const float4*>(Vs + kk * D + qd * 16);
+#pragma unroll
+      for (int c4 = 0; c4 < 4; ++c4) {
+        const float4 vv = vrow[c4];
+        acc[c4 * 4 + 0] = fmaf(pv, vv.x, acc[c4 * 4 + 0]);
+        acc[c4 * 4 + 1] = fmaf(pv, vv.y, acc[c4 * 4 + 1]);
+        acc[c4 * 4 + 2] = fmaf(pv, vv.z, acc[c4 * 4 + 2]);
+        acc[c4 * 4 + 3] = fmaf(pv, vv.w, acc[c4 * 4 + 3]);
+      }
+    }
+    __syncthreads();
+  }
+
+  if (row_ok) {
+    const float inv = 1.f / l;
+    float* orow = p.o + (size_t(bh) * p.Nq + row) * D + qd * 16;
+#pragma unroll
+    for (int c4 = 0; c4 < 4; ++c4)
+      *reinterpret_cast<float4*>(orow + c4 * 4) =
+          make_float4(acc[c4 * 4] * inv, acc[c4 * 4 + 1] * inv, acc[c4 * 4 + 2] * inv, acc[c4 * 4 + 3] * inv);
+    if (qd == 0) p.lse[size_t(bh) * p.Nq + row] = m + logf(l);
+  }
+}
+
+}  // namespace fa

@@ -1,0 +1,159 @@
+/*
+ * fa.h — C ABI of the B200 (sm_100a) exact-attention library.
+ *
+ * The operation is exact scaled-dot-product attention, O = softmax(Q K^T * scale) V,
+ * computed tile by tile with the online-softmax recurrence (running maximum m, sum
+ * l = sum_j e^{s_j - m}, numerator u = sum_j e^{s_j - m} v_j; l and u rescaled by
+ * e^{m - m'} whenever a tile raises the maximum; output u / l), so the Nq x Nkv score
+ * matrix never reaches device memory.
+ *   - Definition: "Autoatención, kernels CUDA y FlashAttention", §1 (Scores = QK^T /
+ *     sqrt(d_k); row softmax; Attention(Q,K,V) = softmax(QK^T / sqrt(d_k)) V; heads in
+ *     parallel).
+ *   - Blocked evaluation and recomputation in the backward pass: same page, §3
+ *     ("Procesamiento por bloques", "El truco de Softmax en línea", "Recálculo durante
+ *     la retropropagación").
+ *   - The (m, l, u) recurrence and why block results cannot be averaged: "FlashAttention"
+ *     (paweldubiel.com notes), "No basta con promediar los resultados de los bloques".
+ *   - GQA: same page, "Mecanismo y detalles", last paragraph.
+ *   - Paged KV cache and block table: "Kernels de atención rápida y fusión de operadores"
+ *     (the-ai.news), "Atención tipo FlashAttention y atención paginada".
+ *
+ * Conventions common to every entry point
+ *   - All tensor pointers are DEVICE pointers to contiguous row-major arrays, at least
+ *     16-byte aligned.  The caller owns every buffer, workspaces included; the library
+ *     never allocates device memory and keeps no state between calls.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL is the
+ *     legacy default stream).  FA_OK means the launch was accepted.  Faults that
+ *     happen while the kernel runs surface at the caller's next synchronisation.
+ *   - Arguments are validated on the host before anything is launched.  Nothing is
+ *     launched when a call returns an error.  There is no CPU fallback and no
+ *     alternative backend: unsupported input is an error (FA_ERR_UNSUPPORTED).
+ *   - Layouts: q, o [B, Hq, Nq, d]; k, v [B, Hkv, Nkv, d]; lse [B, Hq, Nq] fp32.
+ *     Query head h reads key/value head h / (Hq / Hkv) (GQA, contiguous groups).
+ *   - lse = m + ln(l) of the scaled scores (natural log), one per query row.
+ *   - Causal masking is bottom-right aligned: query i may attend keys
+ *     j <= i + (Nkv - Nq).  causal with Nq > Nkv is rejected.
+ *   - Every waiting loop inside the kernels is bounded; a wait that runs out sets a
+ *     device status word (read with fa_device_status) and the kernel returns early.
+ */
+#ifndef FA_H_
+#define FA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1,   /* null pointer, non-positive size, misalignment, bad shape */
+  FA_ERR_UNSUPPORTED = 2,   /* valid but not built: head dim, dtype, block size */
+  FA_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed at launch time */
+  FA_ERR_WORKSPACE = 4,     /* workspace missing or smaller than the size query says */
+  FA_ERR_DEVICE_TIMEOUT = 5 /* a bounded in-kernel wait ran out (see fa_device_status) */
+} fa_status;
+
+typedef enum { FA_DTYPE_F32 = 0, FA_DTYPE_BF16 = 1 } fa_dtype;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* fa_status_string(fa_status s);
+
+/* Library version as an integer (major*10000 + minor*100 + patch). */
+int fa_version(void);
+
+/*
+ * fa_fwd — forward pass.  Writes O (dtype `dtype`) and lse (fp32).
+ *   q [B,Hq,Nq,d], k and v [B,Hkv,Nkv,d], o [B,Hq,Nq,d]: dtype `dtype`.
+ *   lse [B,Hq,Nq] fp32, may not be NULL.
+ *   d in {64, 128}.  dtype BF16: tcgen05 tensor-core kernel, fp32 accumulation, P
+ *   rounded to bf16 before P·V.  dtype F32: fp32 SIMT kernel (d == 64 only).
+ *   scale > 0 (usually 1/sqrt(d)); causal 0 or 1.
+ * Errors: FA_ERR_INVALID_ARG (null/misaligned pointer, size <= 0, Hq % Hkv != 0,
+ * scale not finite or <= 0, causal && Nq > Nkv); FA_ERR_UNSUPPORTED (other d or dtype).
+ */
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                 int B, int Hq, int Hkv, int Nq, int Nkv, int d, float scale, int causal,
+                 fa_dtype dtype, void* stream);
+
+/*
+ * fa_bwd_workspace_size — bytes of device workspace fa_bwd needs: an fp32 dQ
+ * accumulator [B,Hq,Nq,d] and the per-row D_i = sum_c dO_ic O_ic [B,Hq,Nq], each
+ * region 256-byte aligned.  Returns 0 for invalid sizes.
+ */
+size_t fa_bwd_workspace_size(int B, int Hq, int Nq, int d);
+
+/*
+ * fa_bwd — backward pass of fa_fwd, recomputing the score tiles from lse instead of
+ * storing them ("Recálculo durante la retropropagación").
+ *   q, k, v, o, dO: dtype `dtype` (BF16 only), layouts as in fa_fwd; lse from fa_fwd.
+ *   dq [B,Hq,Nq,d], dk and dv [B,Hkv,Nkv,d] of dtype `grad_dtype` (F32 or BF16); dk
+ *   and dv are summed over the Hq/Hkv query heads that share a key/value head.
+ *   workspace: at least fa_bwd_workspace_size(B,Hq,Nq,d) bytes, 256-byte aligned;
+ *   its contents on entry do not matter.
+ *   d == 64 or 128.
+ * Errors: as fa_fwd, plus FA_ERR_WORKSPACE.
+ */
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                 const void* dO, void* dq, void* dk, void* dv, fa_dtype grad_dtype,
+                 int B, int Hq, int Hkv, int Nq, int Nkv, int d, float scale, int causal,
+                 fa_dtype dtype, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * fa_paged_decode_workspace_size — bytes of device workspace fa_paged_decode needs
+ * for the split-KV partial results (fp32 O and lse per split) and per-(request,
+ * key/value head) completion counters.  Returns 0 for invalid sizes.
+ */
+size_t fa_paged_decode_workspace_size(int R, int Hq, int d, int max_blocks_per_seq, int block_size);
+
+/*
+ * fa_paged_decode — one decode step over a paged KV cache ("Atención tipo
+ * FlashAttention y atención paginada": a block table links logical positions to
+ * fixed-size physical blocks, and the kernel translates every position through it).
+ *   q [R,Hq,d] bf16: one new query token per request.
+ *   k_cache, v_cache [num_blocks, Hkv, block_size, d] bf16.
+ *   block_table [R, max_blocks_per_seq] int32: logical block -> physical block.
+ *     Entries at or past ceil(ctx_lens[r] / block_size) are never read.
+ *   ctx_lens [R] int32 (device): cached tokens of request r, 1 <= ctx <=
+ *     max_blocks_per_seq * block_size.  The query attends to all of them.
+ *   o [R,Hq,d] bf16.  lse [R,Hq] fp32 or NULL.
+ *   d == 128, block_size == 16.
+ *   A physical block id outside [0, num_blocks) or a ctx_len out of range is not
+ *   dereferenced: the kernel skips it and sets the device status word
+ *   (FA_ERR_INVALID_ARG), so the result for that request is undefined.
+ * Errors: FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_WORKSPACE.
+ */
+fa_status fa_paged_decode(const void* q, const void* k_cache, const void* v_cache,
+                          const int* block_table, const int* ctx_lens, void* o, float* lse,
+                          int R, int Hq, int Hkv, int d, int block_size, int max_blocks_per_seq,
+                          int num_blocks, float scale, fa_dtype dtype,
+                          void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * fa_device_status — synchronises the current device and returns the device status
+ * word the kernels set when a bounded wait runs out (FA_ERR_DEVICE_TIMEOUT) or a
+ * block-table entry is out of range (FA_ERR_INVALID_ARG); FA_OK if none.  With
+ * reset != 0 the word is cleared afterwards.
+ */
+fa_status fa_device_status(int reset);
+
+/*
+ * fa_set_wait_limit_ns — upper bound, in nanoseconds, on every in-kernel wait
+ * launched after this call (default 2e8 ns = 200 ms).  Values < 1000 are clamped to 1000.
+ */
+void fa_set_wait_limit_ns(uint64_t ns);
+
+/*
+ * fa_selftest_wait_timeout — launches a one-CTA kernel that waits, with the current
+ * limit, on a shared-memory barrier that nothing completes, so the wait must run
+ * out.  Returns FA_OK if the launch succeeded; the kernel then sets the device status
+ * word to FA_ERR_DEVICE_TIMEOUT, which fa_device_status reports.  For tests of the
+ * timeout path; never faults or hangs the device.
+ */
+fa_status fa_selftest_wait_timeout(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FA_H_ */

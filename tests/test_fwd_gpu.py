@@ -1,0 +1,149 @@
+"""Forward parity: CUDA kernels vs the fp64 oracle on the same seeded inputs."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import exact_attention_128_b200 as fa
+from exact_attention_128_b200.workloads import (GQA_PREFILL_CAUSAL, VIT_BATCHED_BF16, VIT_LAYER_F32, DenseCase,
+                                                prefill_sweep)
+from oracle import attention_fp64 as ora
+from parity import check_bf16, check_f32, check_lse, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+def run(case):
+    q, k, v = case.make()
+    o, lse = fa.fwd(q.cuda(), k.cuda(), v.cuda(), causal=case.causal, scale=case.scale)
+    torch.cuda.synchronize()
+    assert fa.device_status() == 0
+    return q, k, v, o, lse
+
+
+def test_vit_layer_f32_full():
+    q, k, v, o, lse = run(VIT_LAYER_F32)
+    O, L = ora.attention_fwd(q, k, v, VIT_LAYER_F32.scale, False)
+    check_f32(o, O, "O")
+    check_f32(lse, L, "lse")
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_worked_example_through_kernel(dtype):
+    """Scores [0,0,ln3,ln3] with values [0,0,1,1] give 0.75 (two 2-key blocks would average to 0.5)."""
+    q = torch.zeros(1, 1, 1, 64, dtype=dtype)
+    k = torch.zeros(1, 1, 4, 64, dtype=dtype)
+    v = torch.zeros(1, 1, 4, 64, dtype=dtype)
+    q[0, 0, 0, 0] = 1.0
+    k[0, 0, 2:, 0] = 1.0  # q.k = [0,0,1,1]; scale ln3 turns it into [0,0,ln3,ln3]
+    v[0, 0, 2:, 0] = 1.0
+    o, lse = fa.fwd(q.cuda(), k.cuda(), v.cuda(), scale=math.log(3.0))
+    tol = 1e-6 if dtype == torch.float32 else 4e-3
+    assert abs(o[0, 0, 0, 0].item() - 0.75) <= tol
+    assert abs(lse[0, 0, 0].item() - math.log(8.0)) <= 1e-5
+
+
+def test_vit_batched_bf16_full():
+    q, k, v, o, lse = run(VIT_BATCHED_BF16)
+    O, L = ora.attention_fwd(q, k, v, VIT_BATCHED_BF16.scale, False)
+    check_bf16(o, O, "O")
+    check_lse(lse, L, "lse")
+
+
+EDGE = [
+    # B, Hq, Hkv, Nq, Nkv, d, causal, dtype
+    (1, 1, 1, 1, 1, 64, False, "bf16"),
+    (1, 1, 1, 1, 1, 128, True, "bf16"),
+    (1, 2, 1, 127, 127, 64, True, "bf16"),
+    (1, 2, 2, 129, 129, 128, True, "bf16"),
+    (2, 4, 1, 200, 333, 128, False, "bf16"),
+    (1, 6, 6, 256, 256, 64, True, "bf16"),
+    (1, 4, 2, 257, 257, 128, False, "bf16"),
+    (1, 3, 1, 100, 612, 128, True, "bf16"),
+    (1, 2, 1, 513, 513, 64, True, "bf16"),
+    (1, 8, 2, 1000, 1000, 128, True, "bf16"),
+    (1, 2, 1, 1, 300, 128, True, "bf16"),
+    (1, 2, 2, 77, 77, 64, False, "f32"),
+    (1, 4, 2, 130, 200, 64, True, "f32"),
+    (2, 2, 1, 1, 65, 64, False, "f32"),
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Nq,Nkv,d,causal,dtype", EDGE)
+def test_edge_shapes(B, Hq, Hkv, Nq, Nkv, d, causal, dtype):
+    case = DenseCase("edge", B, Hq, Hkv, Nq, Nkv, d, dtype, causal, 11 + Nq + Nkv)
+    q, k, v, o, lse = run(case)
+    O, L = ora.attention_fwd(q, k, v, case.scale, causal)
+    if dtype == "f32":
+        check_f32(o, O, "O")
+        check_f32(lse, L, "lse")
+    else:
+        check_bf16(o, O, "O")
+        check_lse(lse, L, "lse")
+
+
+def test_causal_row0_returns_v0_exactly():
+    case = DenseCase("row0", 2, 8, 2, 300, 300, 128, "bf16", True, 21)
+    q, k, v, o, lse = run(case)
+    vr = v.repeat_interleave(4, dim=1)
+    assert torch.equal(o[:, :, 0].cpu(), vr[:, :, 0])
+
+
+def _sample_rows(n, rng, extra=20):
+    fixed = [0, 1, 127, 128, 255, 256, 257, n // 2, n - 129, n - 128, n - 2, n - 1]
+    rows = set(r for r in fixed if 0 <= r < n)
+    rows.update(int(x) for x in rng.choice(n, size=min(n, extra), replace=False))
+    return sorted(rows)
+
+
+def test_gqa_prefill_causal_full_size():
+    """B=4, Hq=32, Hkv=8, N=8192, d=128, causal: every head on sampled rows, two heads in full."""
+    case = GQA_PREFILL_CAUSAL
+    q, k, v, o, lse = run(case)
+    rng = np.random.default_rng(3)
+    on, ln = to_np(o), lse.cpu().numpy()
+    for b in range(case.B):
+        for h in range(case.Hq):
+            rows = _sample_rows(case.Nq, rng, 8)
+            O, L = ora.attention_fwd_rows(q, k, v, case.scale, True, b, h, rows)
+            assert np.abs(on[b, h, rows] - O).max() <= 2e-2
+            assert np.abs(ln[b, h, rows] - L).max() <= 1e-3
+    for b, h in ((0, 0), (3, 31)):
+        for r0 in range(0, case.Nq, 2048):
+            rows = list(range(r0, r0 + 2048))
+            O, L = ora.attention_fwd_rows(q, k, v, case.scale, True, b, h, rows)
+            check_bf16(o[b, h, r0 : r0 + 2048], O, f"O[{b},{h}]")
+            check_lse(lse[b, h, r0 : r0 + 2048], L, "lse")
+
+
+@pytest.mark.parametrize("case", prefill_sweep(), ids=lambda c: c.name)
+def test_noncausal_sweep_sampled(case):
+    q, k, v, o, lse = run(case)
+    rng = np.random.default_rng(case.seed)
+    for b, h in ((0, 0), (case.B - 1, case.Hq - 1), (case.B // 2, 13)):
+        rows = _sample_rows(case.Nq, rng, 24)
+        O, L = ora.attention_fwd_rows(q, k, v, case.scale, False, b, h, rows)
+        check_bf16(o[b, h, rows], O, f"{case.name} O[{b},{h}]")
+        check_lse(lse[b, h, rows], L, "lse")
+
+
+def test_repeat_calls_are_identical():
+    case = DenseCase("repeat", 1, 4, 1, 640, 640, 128, "bf16", True, 31)
+    q, k, v = (t.cuda() for t in case.make())
+    o1, l1 = fa.fwd(q, k, v, causal=True)
+    o2, l2 = fa.fwd(q, k, v, causal=True)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_wait_timeout_sets_status_without_fault():
+    fa.device_status(reset=True)
+    fa.set_wait_limit_ns(2_000_000)
+    try:
+        fa.selftest_wait_timeout()
+        assert fa.device_status(reset=True) == fa.FA_ERR_DEVICE_TIMEOUT
+    finally:
+        fa.set_wait_limit_ns(200_000_000)
+    # the context is still usable
+    x = torch.ones(4, device="cuda")
+    assert x.sum().item() == 4.0
