@@ -430,6 +430,8 @@ def main():
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--only", choices=["prefill_causal", "prefill_noncausal", "train", "decode"],
+                    help="measure just this one secondary workload (for profiling runs) and print it")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -456,6 +458,21 @@ def main():
     dev = torch.device("cuda", local)
     fa.lib()
     fa.device_status(reset=True)
+
+    if args.only:
+        if args.only == "train":
+            r = measure_train(W.TRAIN_CAUSAL, dev, args.steps, args.warmup, world, peaks)
+        elif args.only == "decode":
+            r = measure_decode(W.PAGED_DECODE, dev, args.steps, args.warmup, world, peaks)
+        else:
+            c = W.GQA_PREFILL_CAUSAL if args.only == "prefill_causal" else W.prefill_sweep()[3]
+            r = measure_dense_fwd(c, dev, args.steps, args.warmup, world, peaks)
+        r.pop("rot_bytes", None)
+        if rank == 0:
+            print(json.dumps({"only": args.only, "steps": args.steps, **r}))
+        if fa.device_status(reset=True) != 0:
+            raise SystemExit("device status set after the run")
+        return
 
     sampler = ClockSampler(local)
     sampler.start()
