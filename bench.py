@@ -49,24 +49,28 @@ def load_peaks():
         return FALLBACK, "fallback"
 
 
-def kernel_sources_sha() -> str:
+def kernel_sources_sha(files) -> str:
+    """Hash of the kernel source files a profile was taken on (csrc-relative names)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "exact_attention_128_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    for f in sorted(files):
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
 
 
 def traffic_for(kernel: str):
-    """Per-launch DRAM bytes from a committed ncu summary, if taken on the current sources."""
+    """Per-launch DRAM bytes (read + write) from a committed ncu summary.
+
+    None unless the summary was taken on the current sources of that kernel.
+    """
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
             t = json.load(f)
     except (OSError, ValueError):
         return None
     e = t.get(kernel)
-    if not e or e.get("src_sha") != kernel_sources_sha():
+    if not e or e.get("src_sha") != kernel_sources_sha(e.get("files", [])):
         return None
     return e.get("bytes_per_launch")
 
@@ -155,9 +159,15 @@ def max_over_ranks(x: float, world: int) -> float:
     import torch
     import torch.distributed as dist
 
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(units_per_step_per_rank: float, steps: int, max_ms: float, world: int) -> float:
+    """Whole-job rate: every rank processes its own replica; the slowest rank's time counts."""
+    return world * units_per_step_per_rank * steps / (max_ms * 1e-3)
 
 
 def n_rotations(bytes_per_set: int) -> int:
@@ -515,7 +525,7 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_oracle_dense(case, budget_s=12.0)
 
-    value = world * case.fwd_flops() * args.steps / (head["ms"] * 1e-3) / 1e12
+    value = job_throughput(case.fwd_flops(), args.steps, head["ms"], world) / 1e12
     line = {
         "metric": METRIC,
         "value": round(value, 3),
