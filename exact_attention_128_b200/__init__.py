@@ -49,6 +49,7 @@ EXPORTED = {
     "fa_bwd": (_i, [_vp] * 9 + [_i] + [_i] * 6 + [_f, _i, _i, _vp, _sz, _vp]),
     "fa_paged_decode_workspace_size": (_sz, [_i] * 5),
     "fa_paged_decode": (_i, [_vp] * 7 + [_i] * 7 + [_f, _i, _vp, _sz, _vp]),
+    "fa_paged_decode_noalloc": (_i, [_vp] * 7 + [_i] * 7 + [_f, _i, _vp]),
     "fa_device_status": (_i, [_i]),
     "fa_set_wait_limit_ns": (None, [ctypes.c_uint64]),
     "fa_selftest_wait_timeout": (_i, [_vp]),

@@ -222,3 +222,56 @@ fa_status fa_paged_decode(const void* q, const void* k_cache, const void* v_cach
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------------
+// Paged decode without a caller workspace.
+//
+// Some callers cannot call cudaMalloc: plugins hosted inside a framework that owns
+// every device allocation and offers its kernels no workspace, and latency-critical
+// serving loops that must not allocate after start-up (cudaMalloc may synchronise the
+// device and takes an unbounded time).  fa_paged_decode_noalloc gives them the same
+// decode step with its split-KV scratch in a fixed array that lives in this library's
+// device image: every GPU that loads the library holds FA_NOALLOC_SCRATCH_BYTES of it
+// until the process exits.
+// ------------------------------------------------------------------------------
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[FA_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+void* g_noalloc_ptr[kMaxDevices] = {};
+std::mutex g_noalloc_mu;
+
+// Device address of the scratch array on the current device.  In host code the array's
+// name is only a host-side stand-in, so the address is looked up once per device with
+// that device current, and cached.
+fa_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return FA_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return FA_OK;
+}
+
+}  // namespace
+
+extern "C" fa_status fa_paged_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                                             const int* block_table, const int* ctx_lens, void* o, float* lse,
+                                             int R, int Hq, int Hkv, int d, int block_size, int max_blocks_per_seq,
+                                             int num_blocks, float scale, fa_dtype dtype, void* stream) {
+  const size_t need = fa_paged_decode_workspace_size(R, Hq, d, max_blocks_per_seq, block_size);
+  if (need > size_t(FA_NOALLOC_SCRATCH_BYTES)) return FA_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  // Invalid sizes give need == 0; fa_paged_decode then reports the argument error.
+  if (need > 0) {
+    const fa_status s = noalloc_scratch(&scratch);
+    if (s != FA_OK) return s;
+  }
+  return fa_paged_decode(q, k_cache, v_cache, block_table, ctx_lens, o, lse, R, Hq, Hkv, d, block_size,
+                         max_blocks_per_seq, num_blocks, scale, dtype, scratch, need, stream);
+}

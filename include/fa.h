@@ -131,6 +131,35 @@ fa_status fa_paged_decode(const void* q, const void* k_cache, const void* v_cach
                           void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * fa_paged_decode_noalloc — fa_paged_decode for callers that cannot allocate device
+ * memory.  (No counterpart on the pages: this is a deployment variant of the decode
+ * step, not part of the method.)
+ *
+ * Who needs it: code hosted inside a framework that owns all device allocations and
+ * gives its kernels no workspace, and latency-critical loops that must not call
+ * cudaMalloc after start-up (it can synchronise the device and take unbounded time).
+ *
+ * Arguments and results are those of fa_paged_decode minus the workspace: the split-KV
+ * partials go to a fixed scratch array compiled into the library, FA_NOALLOC_SCRATCH_BYTES
+ * (8 MiB) on every GPU that loads the library, held until the process exits.  Calls
+ * whose fa_paged_decode_workspace_size(R, Hq, d, max_blocks_per_seq, block_size) exceeds
+ * that limit are rejected with FA_ERR_WORKSPACE before anything is launched.  The
+ * function never calls cudaMalloc, cudaFree or any allocating library routine.
+ *
+ * The first call on a device (with that device current) looks up the scratch array's
+ * device address and caches it; make that first call before any stream capture.  Every
+ * call shares the one array, which keeps the last call's contents; nothing in it has to
+ * start at zero (each partial the merge reads is written earlier in the same call).
+ * Calls that overlap on the GPU (different streams, or different host threads without
+ * ordering between them) race on the array and give undefined results.
+ */
+#define FA_NOALLOC_SCRATCH_BYTES (8u * 1024u * 1024u)
+fa_status fa_paged_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                                  const int* block_table, const int* ctx_lens, void* o, float* lse,
+                                  int R, int Hq, int Hkv, int d, int block_size, int max_blocks_per_seq,
+                                  int num_blocks, float scale, fa_dtype dtype, void* stream);
+
+/*
  * fa_device_status — synchronises the current device and returns the device status
  * word the kernels set when a bounded wait runs out (FA_ERR_DEVICE_TIMEOUT) or a
  * block-table entry is out of range (FA_ERR_INVALID_ARG); FA_OK if none.  With
