@@ -1,13 +1,450 @@
-// bwd_bf16.cuh — backward pass (placeholder until the tensor-core kernel lands).
+// bwd_bf16.cuh — backward pass of exact attention on the 5th-generation tensor cores.
+//
+// "Autoatención, kernels CUDA y FlashAttention" §3 ("Recálculo durante la
+// retropropagación") and "FlashAttention" (paweldubiel.com notes, "Mecanismo y
+// detalles"): the forward pass keeps only small per-row normalisation statistics (here
+// lse = m + ln l) and the backward pass recomputes the attention tiles on chip instead
+// of reading an N x N matrix back from memory.  The gradients themselves are not on the
+// pages; they are those of the definition O = softmax(S) V, S = scale Q K^T:
+//     P = exp(S - lse),  dV = P^T dO,  dP = dO V^T,  D_i = sum_c dO_ic O_ic,
+//     dS = P * (dP - D),  dQ = scale dS K,  dK = scale dS^T Q.
+//
+// Three kernels:
+//   1. fa_bwd_preprocess_kernel: D_i, lse in base 2 (padded to whole 128-row tiles with
+//      +inf, so padded rows get P = 0), and zeroes the fp32 dQ accumulator.
+//   2. fa_bwd_bf16_kernel: one CTA per (128-key tile j, batch, key/value head).  It keeps
+//      K_j, V_j in shared memory and walks the G query heads of its group and their
+//      query tiles i (causal: only tiles at or below the diagonal):
+//        warp 0      TMA producer: K_j, V_j once; Q_i, dO_i, lse_i, D_i per step (2 stages)
+//        warp 1      MMA issuer (one thread): S^T = K_j Q_i^T and dP^T = V_j dO_i^T into
+//                    TMEM; then dV += P^T dO_i and dK += dS^T Q_i with P^T, dS^T read from
+//                    TMEM, and dQ_i = dS K_j with dS read from shared memory.
+//        warps 4-7   one thread per key (TMEM lane): P^T and dS^T from S^T, dP^T, lse, D;
+//                    P^T and dS^T (bf16) go back over S^T and dP^T in TMEM, dS^T also to
+//                    shared memory (swizzled, query-major) for the dQ MMA.  At the end
+//                    they write dK_j and dV_j.
+//        warps 8-11  one thread per query row: read dQ_i from TMEM and add it into the fp32
+//                    accumulator with vector reductions (red.global.add.v4.f32).
+//   3. fa_bwd_finalize_kernel: fp32 dQ accumulator -> bf16 dq (only for bf16 gradients;
+//      fp32 gradients accumulate straight into dq).
+//
+// The scale is folded into dS before it is rounded to bf16, so dK and dQ need no
+// further scaling.  TMEM (512 columns): S^T [0,128), dP^T [128,256), dV, dK (D columns
+// each), and dQ: two buffers of D columns when D = 64, or (D = 128) the dP^T columns,
+// which are free once dK has consumed dS^T.
 #pragma once
 #include "common.cuh"
 
 namespace fa {
 
-inline fa_status bwd_launch(const void*, const void*, const void*, const void*, const float*, const void*, void*,
-                            void*, void*, fa_dtype, int, int, int, int, int, int, float, int, void*, cudaStream_t,
-                            uint64_t) {
-  return FA_ERR_UNSUPPORTED;
+template <int D>
+struct BwdCfg {
+  static constexpr int BM = 128;  // query rows per step
+  static constexpr int BN = 128;  // keys per CTA
+  static constexpr int KB = D / 64;
+  static constexpr int TILE = 128 * D * 2;  // one [128 x D] bf16 tile
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = OFF_K + TILE;
+  static constexpr int OFF_Q = OFF_V + TILE;           // + stage * TILE
+  static constexpr int OFF_DO = OFF_Q + 2 * TILE;      // + stage * TILE
+  static constexpr int OFF_DS = OFF_DO + 2 * TILE;     // [2 query chunks][128 keys][128 B]
+  static constexpr int OFF_STAT = OFF_DS + 128 * 128 * 2;  // per stage: lse2[128], D[128]
+  static constexpr int OFF_BAR = OFF_STAT + 2 * 2 * 512;
+  // D = 128 fills the 227 KB limit exactly, leaving no room to re-align the base: that
+  // variant relies on the dynamic shared memory starting 1024-byte aligned and checks it.
+  static constexpr int SLACK = (D == 128) ? 0 : 1024;
+  static constexpr int SMEM = OFF_BAR + 256 + SLACK;
+  static constexpr int THREADS = 384;
+  static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DV = 256, COL_DK = 256 + D;
+  static constexpr int NQB = (D == 64) ? 2 : 1;  // dQ TMEM buffers
+  __host__ __device__ static constexpr uint32_t col_dq(int buf) { return D == 64 ? uint32_t(384 + 64 * buf) : COL_DP; }
+};
+
+struct BwdParams {
+  float* dq_acc;          // fp32 [B,Hq,Nq,D] (the caller's dq when gradients are fp32)
+  const float* lse2;      // [B*Hq][Nq_pad] lse * log2(e), +inf past Nq
+  const float* dstat;     // [B*Hq][Nq_pad] D_i, 0 past Nq
+  void* dk;
+  void* dv;
+  int grad_bf16;
+  int Hq, Hkv, Nq, Nkv, Nq_pad;
+  float scale;
+  float scale_log2;
+  uint64_t wait_ns;
+};
+
+struct BwdBars {
+  uint64_t kv_full;
+  uint64_t qdo_full[2];
+  uint64_t qdo_empty[2];
+  uint64_t sdp_full;
+  uint64_t ds_ready;
+  uint64_t dq_full[2];
+  uint64_t dq_free[2];
+  uint64_t dkdv_full;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(smem_dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
+
+// ------------------------------------------------------------------------------ 1
+// D_i = sum_c dO_ic O_ic per query row; lse2 = lse * log2(e); both padded to Nq_pad.
+// 8 threads per row, each covering D/8 consecutive elements.
+template <int D>
+__global__ void __launch_bounds__(256) fa_bwd_preprocess_kernel(const __nv_bfloat16* o, const __nv_bfloat16* dO,
+                                                                 const float* lse, float* lse2, float* dstat,
+                                                                 float* dq_zero, long total_rows_pad, int Nq,
+                                                                 int Nq_pad, long dq_elems) {
+  const long gt = long(blockIdx.x) * blockDim.x + threadIdx.x;
+  const long row = gt >> 3;  // padded row index
+  const int part = int(gt & 7);
+  if (row < total_rows_pad) {
+    const long bh = row / Nq_pad;
+    const int q = int(row % Nq_pad);
+    float acc = 0.f;
+    if (q < Nq) {
+      const size_t base = (size_t(bh) * Nq + q) * D + part * (D / 8);
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c) {
+        const uint4 a = *reinterpret_cast<const uint4*>(o + base + c * 8);
+        const uint4 g = *reinterpret_cast<const uint4*>(dO + base + c * 8);
+        const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
+        const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&g);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 fa = __bfloat1622float2(a2[e]), fg = __bfloat1622float2(g2[e]);
+          acc = fmaf(fa.x, fg.x, acc);
+          acc = fmaf(fa.y, fg.y, acc);
+        }
+      }
+    }
+    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+    acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+    acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+    if (part == 0) {
+      dstat[row] = q < Nq ? acc : 0.f;
+      lse2[row] = q < Nq ? lse[size_t(bh) * Nq + q] * 1.4426950408889634f : INFINITY;
+    }
+  }
+  // zero the fp32 dQ accumulator (grid-stride, float4)
+  const long n4 = dq_elems / 4;
+  for (long i = gt; i < n4; i += long(gridDim.x) * blockDim.x)
+    reinterpret_cast<float4*>(dq_zero)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+// ------------------------------------------------------------------------------ 3
+__global__ void __launch_bounds__(256) fa_bwd_finalize_kernel(const float* acc, __nv_bfloat16* dq, long n) {
+  const long i = (long(blockIdx.x) * blockDim.x + threadIdx.x) * 4;
+  if (i < n) {
+    const float4 v = *reinterpret_cast<const float4*>(acc + i);
+    uint2 pk;
+    pk.x = pack_bf16x2(v.x, v.y);
+    pk.y = pack_bf16x2(v.z, v.w);
+    *reinterpret_cast<uint2*>(dq + i) = pk;
+  }
+}
+
+// ------------------------------------------------------------------------------ 2
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(384, 1)
+    fa_bwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                       const BwdParams p) {
+  // tmO maps dO (same geometry as Q)
+  using C = BwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  if (C::SLACK == 0 && (smem_u32(smem_raw) & 1023u) != 0) {  // uniform across the CTA
+    if (threadIdx.x == 0) set_status(FA_ERR_UNSUPPORTED, 299);
+    return;
+  }
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  BwdBars* bars = reinterpret_cast<BwdBars*>(smem + C::OFF_BAR);
+  volatile int* abort_flag = &bars->abort_flag;
+
+  const int warp = warp_id(), lane = lane_id();
+  const int j = blockIdx.x;  // key tile (low j = most causal work: scheduled first)
+  const int bk = blockIdx.y;
+  const int b = bk / p.Hkv, hk = bk % p.Hkv;
+  const int G = p.Hq / p.Hkv;
+  const int off = p.Nkv - p.Nq;
+  const int k0 = j * C::BN;
+  // first query tile with a row that may see key k0 (row + off >= k0)
+  const int i_begin = CAUSAL ? max(0, k0 - off) / C::BM : 0;
+  const int n_qt = (p.Nq + C::BM - 1) / C::BM;
+  const int n_i = max(0, n_qt - i_begin);
+  const int n_steps = G * n_i;  // step s: head h = hk*G + s / n_i, tile i = i_begin + s % n_i
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->kv_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars->qdo_full[s], 1);
+      mbar_init(&bars->qdo_empty[s], 1);
+      mbar_init(&bars->dq_full[s], 1);
+      mbar_init(&bars->dq_free[s], 4);
+    }
+    mbar_init(&bars->sdp_full, 1);
+    mbar_init(&bars->ds_ready, 4);
+    mbar_init(&bars->dkdv_full, 1);
+    bars->abort_flag = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  const uint32_t sbase = smem_u32(smem);
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0 && n_steps > 0) {
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      prefetch_tmap(&tmO);
+      mbar_arrive_expect_tx(&bars->kv_full, 2 * C::TILE);
+      for (int kb = 0; kb < C::KB; ++kb) {
+        tma_load_3d(smem + C::OFF_K + kb * 128 * 128, &tmK, &bars->kv_full, kb * 64, k0, bk);
+        tma_load_3d(smem + C::OFF_V + kb * 128 * 128, &tmV, &bars->kv_full, kb * 64, k0, bk);
+      }
+      for (int s = 0; s < n_steps; ++s) {
+        const int st = s & 1;
+        if (s >= 2 && !mbar_wait(&bars->qdo_empty[st], ((s >> 1) - 1) & 1, p.wait_ns, abort_flag, 200)) break;
+        const int h = hk * G + s / n_i, i = i_begin + s % n_i;
+        const int bh = b * p.Hq + h;
+        mbar_arrive_expect_tx(&bars->qdo_full[st], 2 * C::TILE + 1024);
+        for (int kb = 0; kb < C::KB; ++kb) {
+          tma_load_3d(smem + C::OFF_Q + st * C::TILE + kb * 128 * 128, &tmQ, &bars->qdo_full[st], kb * 64,
+                      i * C::BM, bh);
+          tma_load_3d(smem + C::OFF_DO + st * C::TILE + kb * 128 * 128, &tmO, &bars->qdo_full[st], kb * 64,
+                      i * C::BM, bh);
+        }
+        const size_t srow = size_t(bh) * p.Nq_pad + size_t(i) * C::BM;
+        bulk_load(smem + C::OFF_STAT + st * 1024, p.lse2 + srow, 512, &bars->qdo_full[st]);
+        bulk_load(smem + C::OFF_STAT + st * 1024 + 512, p.dstat + srow, 512, &bars->qdo_full[st]);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0 && n_steps > 0) {
+      constexpr uint32_t idKK = idesc_bf16_f32(128, 128, 0);  // S^T, dP^T: both operands K-major
+      constexpr uint32_t idTS = idesc_bf16_f32(128, D, 1);    // dV, dK: B (dO, Q) MN-major
+      constexpr uint32_t idQ = idesc_bf16_f32(128, D, 1) | (1u << 15);  // dQ: A (dS) and B (K) MN-major
+      bool ok = mbar_wait(&bars->kv_full, 0, p.wait_ns, abort_flag, 210);
+      for (int s = 0; s < n_steps && ok; ++s) {
+        const int st = s & 1;
+        ok = mbar_wait(&bars->qdo_full[st], (s >> 1) & 1, p.wait_ns, abort_flag, 211);
+        if (!ok) break;
+        if constexpr (D == 128) {  // dP^T overwrites the previous dQ: wait for its drain
+          if (s > 0 && !(ok = mbar_wait(&bars->dq_free[0], (s - 1) & 1, p.wait_ns, abort_flag, 212))) break;
+        }
+        tc_fence_after();
+        const uint32_t sQ = sbase + C::OFF_Q + st * C::TILE, sO = sbase + C::OFF_DO + st * C::TILE;
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint32_t koff = (ks >> 2) * 128 * 128 + (ks & 3) * 32;
+          mma_ss(tmem + C::COL_S, sdesc_sw128(sbase + C::OFF_K + koff, 16, 1024), sdesc_sw128(sQ + koff, 16, 1024),
+                 idKK, ks > 0);
+        }
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint32_t koff = (ks >> 2) * 128 * 128 + (ks & 3) * 32;
+          mma_ss(tmem + C::COL_DP, sdesc_sw128(sbase + C::OFF_V + koff, 16, 1024), sdesc_sw128(sO + koff, 16, 1024),
+                 idKK, ks > 0);
+        }
+        mma_commit(&bars->sdp_full);
+        ok = mbar_wait(&bars->ds_ready, s & 1, p.wait_ns, abort_flag, 213);
+        if (!ok) break;
+        tc_fence_after();
+        // dV += P^T dO ; dK += dS^T Q  (K dimension = the 128 queries of the step)
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint32_t acc = (s > 0 || ks > 0) ? 1u : 0u;
+          mma_ts(tmem + C::COL_DV, tmem + C::COL_S + ks * 8, sdesc_sw128(sO + ks * 2048, 128 * 128, 1024), idTS,
+                 acc);
+          mma_ts(tmem + C::COL_DK, tmem + C::COL_DP + ks * 8, sdesc_sw128(sQ + ks * 2048, 128 * 128, 1024), idTS,
+                 acc);
+        }
+        const int qb = (C::NQB == 2) ? (s & 1) : 0;
+        if constexpr (D == 64) {
+          if (s >= 2 && !(ok = mbar_wait(&bars->dq_free[qb], ((s >> 1) - 1) & 1, p.wait_ns, abort_flag, 214)))
+            break;
+        }
+        // dQ_i = dS K_j  (M = queries, K dimension = the 128 keys)
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+          mma_ss(tmem + C::col_dq(qb), sdesc_sw128(sbase + C::OFF_DS + ks * 2048, 128 * 128, 1024),
+                 sdesc_sw128(sbase + C::OFF_K + ks * 2048, 128 * 128, 1024), idQ, ks > 0);
+        mma_commit(&bars->dq_full[qb]);
+        mma_commit(&bars->qdo_empty[st]);
+      }
+      if (ok) mma_commit(&bars->dkdv_full);
+    }
+  } else if (warp >= 4 && warp < 8) {
+    // ---------------------------------------------------------------- softmax-gradient (key rows)
+    const int wq = warp & 3;
+    const int r = wq * 32 + lane;  // key within the tile == TMEM lane
+    const int key = k0 + r;
+    const uint32_t lane_off = uint32_t(wq * 32) << 16;
+    const float sl2 = p.scale_log2, scale = p.scale;
+    bool ok = true;
+    for (int s = 0; s < n_steps && ok; ++s) {
+      const int st = s & 1;
+      const int i = i_begin + s % n_i;
+      ok = warp_wait(&bars->sdp_full, s & 1, p.wait_ns, abort_flag, 220) &&
+           warp_wait(&bars->qdo_full[st], (s >> 1) & 1, p.wait_ns, abort_flag, 221);
+      if (!ok) break;
+      tc_fence_after();
+      // columns q < lim are masked for this key (causal); a key past Nkv masks everything
+      int lim = 0;
+      if (key >= p.Nkv) lim = 128;
+      else if (CAUSAL) lim = min(128, max(0, key - off - i * C::BM));
+      const float* lse_s = reinterpret_cast<const float*>(smem + C::OFF_STAT + st * 1024);
+      const float* d_s = lse_s + 128;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t sv[32], dv[32];
+        tmem_ld32(tmem + lane_off + C::COL_S + c * 32, sv);
+        tmem_ld32(tmem + lane_off + C::COL_DP + c * 32, dv);
+        tmem_wait_ld();
+        uint32_t pp[16], pd[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 4) {
+          const float4 l4 = *reinterpret_cast<const float4*>(lse_s + c * 32 + e);
+          const float4 d4 = *reinterpret_cast<const float4*>(d_s + c * 32 + e);
+          const float la[4] = {l4.x, l4.y, l4.z, l4.w}, da[4] = {d4.x, d4.y, d4.z, d4.w};
+          float pv[4], dsv[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            float pr = ex2(fmaf(__uint_as_float(sv[e + u]), sl2, -la[u]));
+            if (c * 32 + e + u < lim) pr = 0.f;
+            pv[u] = pr;
+            dsv[u] = pr * (__uint_as_float(dv[e + u]) - da[u]) * scale;
+          }
+          pp[e / 2] = pack_bf16x2(pv[0], pv[1]);
+          pp[e / 2 + 1] = pack_bf16x2(pv[2], pv[3]);
+          pd[e / 2] = pack_bf16x2(dsv[0], dsv[1]);
+          pd[e / 2 + 1] = pack_bf16x2(dsv[2], dsv[3]);
+        }
+        tmem_st16(tmem + lane_off + C::COL_S + c * 16, pp);
+        tmem_st16(tmem + lane_off + C::COL_DP + c * 16, pd);
+        // dS (query-major, 128-byte swizzle): queries [32c, 32c+32) = four 16-byte units
+        uint8_t* dsrow = smem + C::OFF_DS + (c >> 1) * (128 * 128) + r * 128;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int unit = (c & 1) * 4 + u;
+          *reinterpret_cast<uint4*>(dsrow + ((unit ^ (r & 7)) * 16)) =
+              make_uint4(pd[4 * u], pd[4 * u + 1], pd[4 * u + 2], pd[4 * u + 3]);
+        }
+      }
+      tmem_wait_st();
+      fence_proxy_async_smem();  // dS written by the generic proxy, read by the tensor core
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->ds_ready);
+    }
+    // ---- dK_j, dV_j (scale already folded into dS)
+    if (ok && n_steps > 0) ok = warp_wait(&bars->dkdv_full, 0, p.wait_ns, abort_flag, 222);
+    if (ok && n_steps > 0) {
+      tc_fence_after();
+#pragma unroll 1
+      for (int which = 0; which < 2; ++which) {
+        const uint32_t col = which == 0 ? C::COL_DK : C::COL_DV;
+        void* dst = which == 0 ? p.dk : p.dv;
+        const size_t base = (size_t(bk) * p.Nkv + key) * D;
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tmem + lane_off + col + c * 32, v);
+          tmem_wait_ld();
+          if (key < p.Nkv) {
+            if (p.grad_bf16) {
+              uint4* o4 = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(dst) + base + c * 32);
+#pragma unroll
+              for (int q4 = 0; q4 < 4; ++q4)
+                o4[q4] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * q4]), __uint_as_float(v[8 * q4 + 1])),
+                                    pack_bf16x2(__uint_as_float(v[8 * q4 + 2]), __uint_as_float(v[8 * q4 + 3])),
+                                    pack_bf16x2(__uint_as_float(v[8 * q4 + 4]), __uint_as_float(v[8 * q4 + 5])),
+                                    pack_bf16x2(__uint_as_float(v[8 * q4 + 6]), __uint_as_float(v[8 * q4 + 7])));
+            } else {
+              float4* o4 = reinterpret_cast<float4*>(static_cast<float*>(dst) + base + c * 32);
+#pragma unroll
+              for (int q4 = 0; q4 < 8; ++q4)
+                o4[q4] = make_float4(__uint_as_float(v[4 * q4]), __uint_as_float(v[4 * q4 + 1]),
+                                     __uint_as_float(v[4 * q4 + 2]), __uint_as_float(v[4 * q4 + 3]));
+            }
+          }
+        }
+      }
+    } else if (n_steps == 0 && key < p.Nkv) {
+      // no query row can see these keys: their gradients are zero
+      const size_t base = (size_t(bk) * p.Nkv + key) * D;
+      for (int c = 0; c < D; c += 4) {
+        if (p.grad_bf16) {
+          *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.dk) + base + c) = make_uint2(0, 0);
+          *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.dv) + base + c) = make_uint2(0, 0);
+        } else {
+          *reinterpret_cast<float4*>(static_cast<float*>(p.dk) + base + c) = make_float4(0, 0, 0, 0);
+          *reinterpret_cast<float4*>(static_cast<float*>(p.dv) + base + c) = make_float4(0, 0, 0, 0);
+        }
+      }
+    }
+  } else if (warp >= 8) {
+    // ---------------------------------------------------------------- dQ drain (query rows)
+    const int wq = warp & 3;
+    const int r = wq * 32 + lane;
+    const uint32_t lane_off = uint32_t(wq * 32) << 16;
+    bool ok = true;
+    for (int s = 0; s < n_steps && ok; ++s) {
+      const int qb = (C::NQB == 2) ? (s & 1) : 0;
+      const uint32_t ph = (C::NQB == 2) ? ((s >> 1) & 1) : (s & 1);
+      ok = warp_wait(&bars->dq_full[qb], ph, p.wait_ns, abort_flag, 230);
+      if (!ok) break;
+      tc_fence_after();
+      const int h = hk * G + s / n_i, i = i_begin + s % n_i;
+      const int q = i * C::BM + r;
+      float* dst = p.dq_acc + ((size_t(b) * p.Hq + h) * p.Nq + q) * D;
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tmem + lane_off + C::col_dq(qb) + c * 32, v);
+        tmem_wait_ld();
+        if (q < p.Nq) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 4)
+            red_add_v4(dst + c * 32 + e, __uint_as_float(v[e]), __uint_as_float(v[e + 1]),
+                       __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->dq_free[qb]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
 }
 
 }  // namespace fa

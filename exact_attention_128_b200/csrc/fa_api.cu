@@ -69,6 +69,68 @@ fa_status launch_fwd_bf16(const CUtensorMap& mq, const CUtensorMap& mk, const CU
   return launched();
 }
 
+int round_up(int x, int m) { return (x + m - 1) / m * m; }
+
+template <int D, bool CAUSAL>
+fa_status launch_bwd_kernel(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                            const CUtensorMap& mo, const BwdParams& prm, int B, int Hkv, int Nkv,
+                            cudaStream_t st) {
+  using C = BwdCfg<D>;
+  auto kern = fa_bwd_bf16_kernel<D, CAUSAL>;
+  if (set_smem(kern, C::SMEM) != cudaSuccess) return FA_ERR_CUDA;
+  dim3 grid((Nkv + C::BN - 1) / C::BN, B * Hkv);
+  kern<<<grid, C::THREADS, C::SMEM, st>>>(mq, mk, mv, mo, prm);
+  return launched();
+}
+
+// Backward: preprocess (D, padded lse, zeroed dQ accumulator), the tensor-core kernel,
+// and, for bf16 gradients, the dQ cast.  Workspace: [dQ fp32][lse2 pad][D pad].
+fa_status bwd_launch(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+                     void* dq, void* dk, void* dv, fa_dtype grad_dtype, int B, int Hq, int Hkv, int Nq, int Nkv,
+                     int d, float scale, int causal, void* workspace, cudaStream_t st) {
+  const int Nq_pad = round_up(Nq, 128);
+  const size_t rows = size_t(B) * Hq * Nq;
+  const size_t rows_pad = size_t(B) * Hq * Nq_pad;
+  char* ws = static_cast<char*>(workspace);
+  float* dq_ws = reinterpret_cast<float*>(ws);
+  float* lse2 = reinterpret_cast<float*>(ws + align256(rows * d * 4));
+  float* dstat = reinterpret_cast<float*>(ws + align256(rows * d * 4) + align256(rows_pad * 4));
+  float* dq_acc = grad_dtype == FA_DTYPE_F32 ? static_cast<float*>(dq) : dq_ws;
+
+  const long pre_threads = long(rows_pad) * 8;
+  const int pre_blocks = int((pre_threads + 255) / 256);
+  if (d == 64)
+    fa_bwd_preprocess_kernel<64><<<pre_blocks, 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, lse2, dstat, dq_acc,
+        long(rows_pad), Nq, Nq_pad, long(rows) * d);
+  else
+    fa_bwd_preprocess_kernel<128><<<pre_blocks, 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, lse2, dstat, dq_acc,
+        long(rows_pad), Nq, Nq_pad, long(rows) * d);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+
+  CUtensorMap mq, mk, mv, mo;
+  if (!make_map_bf16(&mq, q, d, Nq, B * Hq, 128) || !make_map_bf16(&mk, k, d, Nkv, B * Hkv, 128) ||
+      !make_map_bf16(&mv, v, d, Nkv, B * Hkv, 128) || !make_map_bf16(&mo, dO, d, Nq, B * Hq, 128))
+    return FA_ERR_CUDA;
+  BwdParams prm{dq_acc, lse2, dstat, dk, dv, grad_dtype == FA_DTYPE_BF16 ? 1 : 0, Hq, Hkv, Nq, Nkv, Nq_pad,
+                scale, scale * 1.4426950408889634f, g_wait_ns};
+  fa_status s;
+  if (d == 64)
+    s = causal ? launch_bwd_kernel<64, true>(mq, mk, mv, mo, prm, B, Hkv, Nkv, st)
+               : launch_bwd_kernel<64, false>(mq, mk, mv, mo, prm, B, Hkv, Nkv, st);
+  else
+    s = causal ? launch_bwd_kernel<128, true>(mq, mk, mv, mo, prm, B, Hkv, Nkv, st)
+               : launch_bwd_kernel<128, false>(mq, mk, mv, mo, prm, B, Hkv, Nkv, st);
+  if (s != FA_OK) return s;
+  if (grad_dtype == FA_DTYPE_BF16) {
+    const long n = long(rows) * d;
+    fa_bwd_finalize_kernel<<<int((n / 4 + 255) / 256), 256, 0, st>>>(dq_ws, static_cast<__nv_bfloat16*>(dq), n);
+    return launched();
+  }
+  return FA_OK;
+}
+
 __global__ void selftest_wait_kernel(uint64_t limit_ns) {
   __shared__ uint64_t bar;
   __shared__ int abort_flag;
@@ -157,7 +219,8 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
 size_t fa_bwd_workspace_size(int B, int Hq, int Nq, int d) {
   if (B <= 0 || Hq <= 0 || Nq <= 0 || d <= 0) return 0;
   const size_t rows = size_t(B) * Hq * Nq;
-  return align256(rows * d * sizeof(float)) + align256(rows * sizeof(float));
+  const size_t rows_pad = size_t(B) * Hq * size_t((Nq + 127) / 128 * 128);
+  return align256(rows * d * sizeof(float)) + 2 * align256(rows_pad * sizeof(float));
 }
 
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
@@ -179,8 +242,8 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   if (long(B) * Hq > 65535) return FA_ERR_UNSUPPORTED;
   const size_t need = fa_bwd_workspace_size(B, Hq, Nq, d);
   if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return FA_ERR_WORKSPACE;
-  return fa::bwd_launch(q, k, v, o, lse, dO, dq, dk, dv, grad_dtype, B, Hq, Hkv, Nq, Nkv, d, scale, causal,
-                        workspace, static_cast<cudaStream_t>(stream), g_wait_ns);
+  return bwd_launch(q, k, v, o, lse, dO, dq, dk, dv, grad_dtype, B, Hq, Hkv, Nq, Nkv, d, scale, causal, workspace,
+                    static_cast<cudaStream_t>(stream));
 }
 
 size_t fa_paged_decode_workspace_size(int R, int Hq, int d, int max_blocks_per_seq, int block_size) {

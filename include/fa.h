@@ -79,8 +79,9 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
 
 /*
  * fa_bwd_workspace_size — bytes of device workspace fa_bwd needs: an fp32 dQ
- * accumulator [B,Hq,Nq,d] and the per-row D_i = sum_c dO_ic O_ic [B,Hq,Nq], each
- * region 256-byte aligned.  Returns 0 for invalid sizes.
+ * accumulator [B,Hq,Nq,d], then lse in base 2 and D_i = sum_c dO_ic O_ic, each
+ * [B,Hq,ceil(Nq/128)*128] fp32; every region 256-byte aligned.  Returns 0 for invalid
+ * sizes.
  */
 size_t fa_bwd_workspace_size(int B, int Hq, int Nq, int d);
 

@@ -1,0 +1,83 @@
+"""Backward parity: CUDA kernels vs the fp64 oracle's gradients on the same seeded inputs.
+
+The GPU backward consumes the GPU forward's O and lse (as a training step would); the
+oracle computes everything from q, k, v, dO in fp64.
+"""
+import numpy as np
+import pytest
+import torch
+
+import exact_attention_128_b200 as fa
+from exact_attention_128_b200.workloads import TRAIN_CAUSAL, DenseCase
+from oracle import attention_fp64 as ora
+from parity import check_bf16, check_bf16_stored, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+def run(case, grad_dtype=torch.float32):
+    q, k, v, do = case.make(with_grad_output=True)
+    qd, kd, vd, dod = (t.cuda() for t in (q, k, v, do))
+    o, lse = fa.fwd(qd, kd, vd, causal=case.causal, scale=case.scale)
+    dq, dk, dv = fa.bwd(qd, kd, vd, o, lse, dod, causal=case.causal, scale=case.scale, grad_dtype=grad_dtype)
+    torch.cuda.synchronize()
+    assert fa.device_status() == 0
+    return (q, k, v, do), (dq, dk, dv)
+
+
+def test_train_causal_full_size_sampled_heads():
+    """B=8, H=16, N=4096, d=64, causal: 8 whole heads (each key/value head's full gradients)."""
+    case = TRAIN_CAUSAL
+    (q, k, v, do), (dq, dk, dv) = run(case)
+    heads = [(0, 0), (7, 15), (3, 5), (1, 9), (5, 2), (6, 11), (2, 14), (4, 7)]
+    rq, rk, rv = ora.attention_bwd(q, k, v, do, case.scale, True, heads=heads)
+    for b, h in heads:
+        check_bf16(dq[b, h], rq[b, h], f"dQ[{b},{h}]")
+        check_bf16(dk[b, h], rk[b, h], f"dK[{b},{h}]")
+        check_bf16(dv[b, h], rv[b, h], f"dV[{b},{h}]")
+
+
+EDGE = [
+    # B, Hq, Hkv, Nq, Nkv, d, causal
+    (1, 1, 1, 1, 1, 64, False),
+    (1, 2, 1, 127, 127, 64, True),
+    (2, 4, 2, 200, 200, 64, False),
+    (1, 4, 1, 300, 300, 64, True),
+    (1, 2, 2, 129, 129, 128, True),
+    (1, 4, 2, 256, 384, 128, False),
+    (1, 3, 1, 100, 612, 64, True),
+    (1, 2, 1, 513, 513, 128, True),
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Nq,Nkv,d,causal", EDGE)
+def test_bwd_edge_shapes(B, Hq, Hkv, Nq, Nkv, d, causal):
+    case = DenseCase("bwd_edge", B, Hq, Hkv, Nq, Nkv, d, "bf16", causal, 70 + Nq + Nkv + d)
+    (q, k, v, do), (dq, dk, dv) = run(case)
+    rq, rk, rv = ora.attention_bwd(q, k, v, do, case.scale, causal)
+    check_bf16(dq, rq, "dQ")
+    check_bf16(dk, rk, "dK")
+    check_bf16(dv, rv, "dV")
+
+
+def test_bwd_bf16_gradients():
+    case = DenseCase("bwd_bf16", 1, 4, 2, 640, 640, 64, "bf16", True, 91)
+    (q, k, v, do), (dq, dk, dv) = run(case, torch.bfloat16)
+    assert dq.dtype == dk.dtype == dv.dtype == torch.bfloat16
+    rq, rk, rv = ora.attention_bwd(q, k, v, do, case.scale, True)
+    over = 0
+    for got, ref, n in ((dq, rq, "dQ"), (dk, rk, "dK"), (dv, rv, "dV")):
+        over += check_bf16_stored(got, ref, n)
+    # the allowance is for a handful of elements next to a rounding midpoint, not a trend
+    assert over <= 1e-3 * (dq.numel() + dk.numel() + dv.numel())
+
+
+def test_bwd_gradient_invariants_on_gpu():
+    """Softmax ignores a common key shift: sum_j dK_j = 0 per head; sum_j dV_j = sum_i dO_i (G=1)."""
+    case = DenseCase("inv", 1, 2, 2, 384, 384, 64, "bf16", True, 93)
+    (q, k, v, do), (dq, dk, dv) = run(case)
+    s_dk = to_np(dk).sum(axis=2)
+    s_dv = to_np(dv).sum(axis=2)
+    s_do = do.double().numpy().sum(axis=2)
+    assert np.abs(s_dk).max() < 0.05
+    assert np.abs(s_dv - s_do).max() < 0.05
