@@ -255,17 +255,36 @@ def e2e_fwd(case, dev, steps, warmup, world):
 
 
 def measure_dense_fwd(case, dev, steps, warmup, world, peaks, peak_key="bf16_tflops"):
+    """Forward kernel throughput; the roofline is whichever of tensor or HBM binds.
+
+    Algorithmic work per launch: 4*d FLOP per allowed (query, key) pair and head; bytes
+    = q, k, v read once + o written once (bf16) + lse (fp32).  The bound is the larger of
+    flops / tensor peak and bytes / HBM peak.
+    """
     fns, sets, host, rot_bytes = dense_fwd_step_fns(case, dev)
     ms = timed_loop(fns, steps, warmup, world)
     flops = case.fwd_flops()
+    q, k, v = host
+    nbytes = 2 * q.numel() * 2 + 2 * k.numel() * 2 + case.B * case.Hq * case.Nq * 4
     per_step_ms = ms / steps
-    tflops = flops / (per_step_ms * 1e-3) / 1e12
+    sec = per_step_ms * 1e-3
+    tflops = flops / sec / 1e12
+    gbs = nbytes / sec / 1e9
     kname = f"fa_fwd_bf16_kernel<{case.d},{str(case.causal).lower()}>"
-    peak = peaks[peak_key]
-    roof = {"bound": "tensor", "achieved": round(tflops, 2), "peak": peak, "unit": "TFLOP/s",
-            "frac": round(tflops / peak, 4), "traffic": traffic_for(kname), "kernel": kname,
-            "peak_kind": peak_key, "frac_of_nominal_2250": round(tflops / NOMINAL_BF16_TFLOPS, 4),
-            "algorithmic_flops_per_launch": flops}
+    t_tensor = flops / (peaks[peak_key] * 1e12)
+    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+    if t_hbm > t_tensor:
+        roof = {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(gbs / peaks["hbm_gbs"], 4), "peak_kind": "hbm_gbs",
+                "frac_of_nominal_8000": round(gbs / NOMINAL_HBM_GBS, 4)}
+    else:
+        roof = {"bound": "tensor", "achieved": round(tflops, 2), "peak": peaks[peak_key], "unit": "TFLOP/s",
+                "frac": round(tflops / peaks[peak_key], 4), "peak_kind": peak_key,
+                "frac_of_nominal_2250": round(tflops / NOMINAL_BF16_TFLOPS, 4)}
+    roof.update({"traffic": traffic_for(kname), "kernel": kname, "algorithmic_flops_per_launch": flops,
+                 "algorithmic_bytes_per_launch": nbytes, "tflops": round(tflops, 2), "gbs": round(gbs, 1),
+                 "tensor_frac": round(tflops / peaks[peak_key], 4),
+                 "hbm_frac": round(gbs / peaks["hbm_gbs"], 4)})
     return {"ms": ms, "per_step_ms": per_step_ms, "tflops": tflops, "roofline": roof, "rot_bytes": rot_bytes,
             "launches_per_step": 1}
 

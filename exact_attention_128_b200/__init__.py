@@ -53,6 +53,7 @@ EXPORTED = {
     "fa_device_status": (_i, [_i]),
     "fa_set_wait_limit_ns": (None, [ctypes.c_uint64]),
     "fa_selftest_wait_timeout": (_i, [_vp]),
+    "fa_selftest_exp2": (_i, [_vp, _vp, _i, _vp]),
 }
 
 

@@ -58,14 +58,24 @@ cudaError_t set_smem(K kernel, int bytes) {
 
 fa_status launched() { return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA; }
 
+// Number of SMs of the current device (persistent grids use one CTA per SM).
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return 0;
+  return n;
+}
+
 template <int D, bool CAUSAL>
 fa_status launch_fwd_bf16(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                          const FwdBf16Params& prm, int B, int Hq, int Nq, cudaStream_t st) {
+                          const FwdBf16Params& prm, int Nq, cudaStream_t st) {
   using C = FwdCfg<D>;
   auto kern = fa_fwd_bf16_kernel<D, CAUSAL>;
   if (set_smem(kern, C::SMEM) != cudaSuccess) return FA_ERR_CUDA;
-  dim3 grid((Nq + 2 * C::BM - 1) / (2 * C::BM), B * Hq);
-  kern<<<grid, C::THREADS, C::SMEM, st>>>(mq, mk, mv, prm);
+  const long items = long((Nq + 2 * C::BM - 1) / (2 * C::BM)) * prm.BH;
+  const int sms = sm_count();
+  if (sms <= 0) return FA_ERR_CUDA;
+  kern<<<int(items < sms ? items : sms), C::THREADS, C::SMEM, st>>>(mq, mk, mv, prm);
   return launched();
 }
 
@@ -131,6 +141,17 @@ fa_status bwd_launch(const void* q, const void* k, const void* v, const void* o,
   return FA_OK;
 }
 
+__global__ void selftest_exp2_kernel(const float* x, float* y, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i + 1 < n) {
+    const float2 r = exp2_fma2(make_float2(x[i], x[i + 1]));
+    y[i] = r.x;
+    y[i + 1] = r.y;
+  } else if (i < n) {
+    y[i] = exp2_fma2(make_float2(x[i], x[i])).x;
+  }
+}
+
 __global__ void selftest_wait_kernel(uint64_t limit_ns) {
   __shared__ uint64_t bar;
   __shared__ int abort_flag;
@@ -179,6 +200,13 @@ fa_status fa_selftest_wait_timeout(void* stream) {
   return launched();
 }
 
+fa_status fa_selftest_exp2(const float* x, float* y, int n, void* stream) {
+  if (!x || !y || n <= 0) return FA_ERR_INVALID_ARG;
+  const int pairs = (n + 1) / 2;
+  selftest_exp2_kernel<<<(pairs + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
+  return launched();
+}
+
 fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Nq,
                  int Nkv, int d, float scale, int causal, fa_dtype dtype, void* stream) {
   if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
@@ -190,6 +218,7 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
     return FA_ERR_INVALID_ARG;
   if (long(B) * Hq > 65535) return FA_ERR_UNSUPPORTED;
+  if (long((Nq + 255) / 256) * B * Hq > 0x7fffffffL) return FA_ERR_UNSUPPORTED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
 
   if (dtype == FA_DTYPE_F32) {
@@ -207,13 +236,13 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   if (!make_map_bf16(&mq, q, d, Nq, B * Hq, 128) || !make_map_bf16(&mk, k, d, Nkv, B * Hkv, 128) ||
       !make_map_bf16(&mv, v, d, Nkv, B * Hkv, 128))
     return FA_ERR_CUDA;
-  FwdBf16Params prm{static_cast<__nv_bfloat16*>(o), lse, Hq, Hkv, Nq, Nkv,
+  FwdBf16Params prm{static_cast<__nv_bfloat16*>(o), lse, B * Hq, Hq, Hkv, Nq, Nkv,
                     scale * 1.4426950408889634f, g_wait_ns};
   if (d == 64)
-    return causal ? launch_fwd_bf16<64, true>(mq, mk, mv, prm, B, Hq, Nq, st)
-                  : launch_fwd_bf16<64, false>(mq, mk, mv, prm, B, Hq, Nq, st);
-  return causal ? launch_fwd_bf16<128, true>(mq, mk, mv, prm, B, Hq, Nq, st)
-                : launch_fwd_bf16<128, false>(mq, mk, mv, prm, B, Hq, Nq, st);
+    return causal ? launch_fwd_bf16<64, true>(mq, mk, mv, prm, Nq, st)
+                  : launch_fwd_bf16<64, false>(mq, mk, mv, prm, Nq, st);
+  return causal ? launch_fwd_bf16<128, true>(mq, mk, mv, prm, Nq, st)
+                : launch_fwd_bf16<128, false>(mq, mk, mv, prm, Nq, st);
 }
 
 size_t fa_bwd_workspace_size(int B, int Hq, int Nq, int d) {

@@ -8,36 +8,50 @@
 // a tile raises the maximum, l and u are rescaled by e^{m - m'} before the tile's own
 // terms are added; the output is u / l.
 //
-// One CTA owns two 128-row query tiles (Q0, Q1) of one (batch, query head) and streams
-// the 128-key tiles of its key/value head (GQA: head h reads h / (Hq/Hkv)).
-//   warp 0      TMA producer: Q0/Q1 once, then K_j and V_j into a ring of stages.
+// Persistent kernel: one CTA per SM walks work items (two 128-row query tiles Q0, Q1 of
+// one (batch, query head)), item = blockIdx.x + k * gridDim.x; causal items are ordered
+// heaviest first.  Each item streams the 128-key tiles of its key/value head (GQA: head
+// h reads h / (Hq/Hkv)).  The K/V ring and the Q buffers run ahead across item
+// boundaries, so loads for the next item overlap the current item's tail and epilogue.
+//   warp 0      TMA producer: Q0/Q1 per item (QBUF buffers), K_j and V_j into a ring.
 //   warp 1      MMA issuer (one thread): S_t = Q_t K_j^T into TMEM (SS MMA), then
 //               u_t += P_t V_j with P_t read from TMEM (TS MMA).
 //   warps 4-7   softmax for Q0, warps 8-11 softmax for Q1: each thread owns one
 //               query row = one TMEM lane; it reads S_t, updates (m, l), writes P_t
-//               (bf16) over S_t in TMEM, and rescales u_t in TMEM when m rose.
+//               (bf16) over S_t in TMEM, rescales u_t in TMEM when m rose, and at the
+//               end of an item writes O = u/l and lse.
 // While one warpgroup runs the softmax of its tile, the tensor core works on the
 // other tile, so the exponentials overlap the MMAs.
 //
 // TMEM columns (512 allocated): S0 [0,128), S1 [128,256), u0 [256,256+D), u1 after.
-// Shared memory: Q0, Q1, then NSTAGE K tiles and NSTAGE V tiles, each stored as
-// D/64 column blocks of [rows x 128 bytes] with the 128-byte swizzle TMA writes
-// and the MMA descriptors expect.
+// Shared memory: QBUF x (Q0, Q1), then NSTAGE K tiles and NSTAGE V tiles, each stored
+// as D/64 column blocks of [rows x 128 bytes] with the 128-byte swizzle TMA writes and
+// the MMA descriptors expect.
 #pragma once
 #include "common.cuh"
 
 namespace fa {
 
+// Bit k set: in unmasked tiles, element pair k of every 8 pairs takes the FMA-pipe
+// exponential (exp2_fma2) instead of the SFU one.  Off by default: measured on B200 with
+// 0x24, 0xA4, 0xAA and 0xB6 (25-50 %), every split was slower than the SFU alone in this
+// kernel (e.g. 1006 vs 845-930 TFLOP/s at N = 8192, d = 128), because the softmax warps
+// are limited by issue slots and latency, not by SFU throughput.
+#ifndef FWD_EMU_PAIRS
+#define FWD_EMU_PAIRS 0x00u
+#endif
+
 template <int D>
 struct FwdCfg {
-  static constexpr int BM = 128;  // rows per query tile (two tiles per CTA)
+  static constexpr int BM = 128;  // rows per query tile (two tiles per item)
   static constexpr int BN = 128;  // keys per tile
   static constexpr int KB = D / 64;
   static constexpr int Q_TILE = BM * D * 2;
   static constexpr int KV_TILE = BN * D * 2;
+  static constexpr int QBUF = (D == 128) ? 1 : 2;
   static constexpr int NSTAGE = (D == 128) ? 2 : 4;
-  static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = 2 * Q_TILE;
+  static constexpr int OFF_Q = 0;  // + qb * 2 * Q_TILE + t * Q_TILE
+  static constexpr int OFF_K = QBUF * 2 * Q_TILE;
   static constexpr int OFF_V = OFF_K + NSTAGE * KV_TILE;
   static constexpr int OFF_BAR = OFF_V + NSTAGE * KV_TILE;
   static constexpr int SMEM = OFF_BAR + 256 + 1024;  // + barriers + alignment slack
@@ -50,13 +64,14 @@ struct FwdCfg {
 struct FwdBf16Params {
   __nv_bfloat16* o;
   float* lse;
-  int Hq, Hkv, Nq, Nkv;
+  int BH, Hq, Hkv, Nq, Nkv;
   float scale_log2;  // scale * log2(e)
   uint64_t wait_ns;
 };
 
 struct FwdBars {
-  uint64_t q_full;
+  uint64_t q_full[2];
+  uint64_t q_empty[2];
   uint64_t k_full[4];
   uint64_t v_full[4];
   uint64_t kv_empty[4];
@@ -78,18 +93,23 @@ __global__ void __launch_bounds__(384, 1)
   volatile int* abort_flag = &bars->abort_flag;
 
   const int warp = warp_id(), lane = lane_id();
-  const int qt = CAUSAL ? int(gridDim.x - 1 - blockIdx.x) : int(blockIdx.x);  // heavy causal tiles first
-  const int bh = blockIdx.y;
-  const int b = bh / p.Hq, h = bh % p.Hq;
-  const int hk = h / (p.Hq / p.Hkv);
-  const int q_row0 = qt * 2 * C::BM;
+  const int n_qp = (p.Nq + 2 * C::BM - 1) / (2 * C::BM);
+  const int n_items = n_qp * p.BH;
   const int off = p.Nkv - p.Nq;  // bottom-right causal alignment
-  int kv_end = p.Nkv;
-  if (CAUSAL) kv_end = min(p.Nkv, min(q_row0 + 2 * C::BM, p.Nq) + off);
-  const int n = (kv_end + C::BN - 1) / C::BN;
+  // item -> (query-tile pair, batch*head); causal items heaviest (last query tiles) first
+  auto item_qt = [&](int it) { return CAUSAL ? n_qp - 1 - it / p.BH : it / p.BH; };
+  auto item_bh = [&](int it) { return it % p.BH; };
+  auto item_ntiles = [&](int qt) {
+    int kv_end = p.Nkv;
+    if (CAUSAL) kv_end = min(p.Nkv, min(qt * 2 * C::BM + 2 * C::BM, p.Nq) + off);
+    return (kv_end + C::BN - 1) / C::BN;
+  };
 
   if (threadIdx.x == 0) {
-    mbar_init(&bars->q_full, 1);
+    for (int q = 0; q < C::QBUF; ++q) {
+      mbar_init(&bars->q_full[q], 1);
+      mbar_init(&bars->q_empty[q], 1);
+    }
     for (int s = 0; s < C::NSTAGE; ++s) {
       mbar_init(&bars->k_full[s], 1);
       mbar_init(&bars->v_full[s], 1);
@@ -122,23 +142,34 @@ __global__ void __launch_bounds__(384, 1)
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
-      mbar_arrive_expect_tx(&bars->q_full, 2 * C::Q_TILE);
-      for (int t = 0; t < 2; ++t)
-        for (int kb = 0; kb < C::KB; ++kb)
-          tma_load_3d(smem + C::OFF_Q + t * C::Q_TILE + kb * C::BM * 128, &tmQ, &bars->q_full, kb * 64,
-                      q_row0 + t * C::BM, bh);
-      const int zkv = b * p.Hkv + hk;
-      for (int j = 0; j < n; ++j) {
-        const int st = j % C::NSTAGE, round = j / C::NSTAGE;
-        if (round > 0 && !mbar_wait(&bars->kv_empty[st], (round - 1) & 1, p.wait_ns, abort_flag, 10)) break;
-        mbar_arrive_expect_tx(&bars->k_full[st], C::KV_TILE);
-        for (int kb = 0; kb < C::KB; ++kb)
-          tma_load_3d(smem + C::OFF_K + st * C::KV_TILE + kb * C::BN * 128, &tmK, &bars->k_full[st], kb * 64,
-                      j * C::BN, zkv);
-        mbar_arrive_expect_tx(&bars->v_full[st], C::KV_TILE);
-        for (int kb = 0; kb < C::KB; ++kb)
-          tma_load_3d(smem + C::OFF_V + st * C::KV_TILE + kb * C::BN * 128, &tmV, &bars->v_full[st], kb * 64,
-                      j * C::BN, zkv);
+      int kv = 0;  // K/V tiles issued so far (ring position)
+      int local = 0;
+      bool ok = true;
+      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++local) {
+        const int qt = item_qt(it), bh = item_bh(it);
+        const int b = bh / p.Hq, h = bh % p.Hq;
+        const int zkv = b * p.Hkv + h / (p.Hq / p.Hkv);
+        const int n = item_ntiles(qt);
+        const int qb = local % C::QBUF, quse = local / C::QBUF;
+        if (quse > 0 && !(ok = mbar_wait(&bars->q_empty[qb], (quse - 1) & 1, p.wait_ns, abort_flag, 11))) break;
+        mbar_arrive_expect_tx(&bars->q_full[qb], 2 * C::Q_TILE);
+        for (int t = 0; t < 2; ++t)
+          for (int kb = 0; kb < C::KB; ++kb)
+            tma_load_3d(smem + C::OFF_Q + (qb * 2 + t) * C::Q_TILE + kb * C::BM * 128, &tmQ, &bars->q_full[qb],
+                        kb * 64, qt * 2 * C::BM + t * C::BM, bh);
+        for (int j = 0; j < n; ++j, ++kv) {
+          const int st = kv % C::NSTAGE, round = kv / C::NSTAGE;
+          if (round > 0 && !(ok = mbar_wait(&bars->kv_empty[st], (round - 1) & 1, p.wait_ns, abort_flag, 10)))
+            break;
+          mbar_arrive_expect_tx(&bars->k_full[st], C::KV_TILE);
+          for (int kb = 0; kb < C::KB; ++kb)
+            tma_load_3d(smem + C::OFF_K + st * C::KV_TILE + kb * C::BN * 128, &tmK, &bars->k_full[st], kb * 64,
+                        j * C::BN, zkv);
+          mbar_arrive_expect_tx(&bars->v_full[st], C::KV_TILE);
+          for (int kb = 0; kb < C::KB; ++kb)
+            tma_load_3d(smem + C::OFF_V + st * C::KV_TILE + kb * C::BN * 128, &tmV, &bars->v_full[st], kb * 64,
+                        j * C::BN, zkv);
+        }
       }
     }
   } else if (warp == 1) {
@@ -146,11 +177,12 @@ __global__ void __launch_bounds__(384, 1)
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16_f32(128, C::BN, 0);  // K-major A (Q) and B (K)
       constexpr uint32_t idPV = idesc_bf16_f32(128, D, 1);     // B (V) is MN-major
-      auto issue_S = [&](int t, int st) {
+      auto issue_S = [&](int qb, int t, int st) {
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const int kb = ks >> 2, kin = ks & 3;
-          const uint64_t a = sdesc_sw128(sQ + t * C::Q_TILE + kb * C::BM * 128 + kin * 32, 16, 1024);
+          const uint64_t a =
+              sdesc_sw128(sQ + (qb * 2 + t) * C::Q_TILE + kb * C::BM * 128 + kin * 32, 16, 1024);
           const uint64_t bd = sdesc_sw128(sK + st * C::KV_TILE + kb * C::BN * 128 + kin * 32, 16, 1024);
           mma_ss(tmem + C::COL_S + t * 128, a, bd, idS, ks > 0 ? 1u : 0u);
         }
@@ -163,116 +195,173 @@ __global__ void __launch_bounds__(384, 1)
                  (j > 0 || ks > 0) ? 1u : 0u);
         }
       };
-      bool ok = mbar_wait(&bars->q_full, 0, p.wait_ns, abort_flag, 20) &&
-                mbar_wait(&bars->k_full[0], 0, p.wait_ns, abort_flag, 21);
-      if (ok) {
+      int kv = 0;  // K/V tiles consumed so far (ring position)
+      int g = 0;   // query-tile steps so far (s_full / p_full phase)
+      int local = 0;
+      bool ok = true;
+      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++local) {
+        const int n = item_ntiles(item_qt(it));
+        const int qb = local % C::QBUF;
+        ok = mbar_wait(&bars->q_full[qb], (local / C::QBUF) & 1, p.wait_ns, abort_flag, 20) &&
+             mbar_wait(&bars->k_full[kv % C::NSTAGE], (kv / C::NSTAGE) & 1, p.wait_ns, abort_flag, 21);
+        if (!ok) break;
         tc_fence_after();
-        issue_S(0, 0);
+        issue_S(qb, 0, kv % C::NSTAGE);
         mma_commit(&bars->s_full[0]);
-        issue_S(1, 0);
+        issue_S(qb, 1, kv % C::NSTAGE);
         mma_commit(&bars->s_full[1]);
-        for (int j = 0; j < n && ok; ++j) {
-          const int st = j % C::NSTAGE;
-          const int st2 = (j + 1) % C::NSTAGE;
+        for (int j = 0; j < n; ++j, ++kv, ++g) {
+          const int st = kv % C::NSTAGE;
+          const int st2 = (kv + 1) % C::NSTAGE;
           const bool more = j + 1 < n;
-          ok = mbar_wait(&bars->v_full[st], (j / C::NSTAGE) & 1, p.wait_ns, abort_flag, 22) &&
-               mbar_wait(&bars->p_full[0], j & 1, p.wait_ns, abort_flag, 23);
+          ok = mbar_wait(&bars->v_full[st], (kv / C::NSTAGE) & 1, p.wait_ns, abort_flag, 22) &&
+               mbar_wait(&bars->p_full[0], g & 1, p.wait_ns, abort_flag, 23);
           if (!ok) break;
           tc_fence_after();
           issue_PV(0, st, j);
           if (more) {
-            ok = mbar_wait(&bars->k_full[st2], ((j + 1) / C::NSTAGE) & 1, p.wait_ns, abort_flag, 24);
+            ok = mbar_wait(&bars->k_full[st2], ((kv + 1) / C::NSTAGE) & 1, p.wait_ns, abort_flag, 24);
             if (!ok) break;
             tc_fence_after();
-            issue_S(0, st2);
+            issue_S(qb, 0, st2);
             mma_commit(&bars->s_full[0]);
           } else {
             mma_commit(&bars->o_final[0]);
           }
-          ok = mbar_wait(&bars->p_full[1], j & 1, p.wait_ns, abort_flag, 25);
+          ok = mbar_wait(&bars->p_full[1], g & 1, p.wait_ns, abort_flag, 25);
           if (!ok) break;
           tc_fence_after();
           issue_PV(1, st, j);
           mma_commit(&bars->kv_empty[st]);
           if (more) {
-            issue_S(1, st2);
+            issue_S(qb, 1, st2);
             mma_commit(&bars->s_full[1]);
           } else {
             mma_commit(&bars->o_final[1]);
+            mma_commit(&bars->q_empty[qb]);  // every S of this item has been issued
           }
         }
       }
     }
   } else if (warp >= 4) {
-    // ---------------------------------------------------------------- softmax
+    // ---------------------------------------------------------------- softmax + epilogue
     const int t = (warp - 4) >> 2;              // which query tile
     const int wq = warp & 3;                    // TMEM lane quarter this warp may access
     const int r = wq * 32 + lane;               // row within the tile == TMEM lane
-    const int row = q_row0 + t * C::BM + r;
     const uint32_t lane_off = uint32_t(wq * 32) << 16;
     const uint32_t tS = tmem + lane_off + C::COL_S + t * 128;
     const uint32_t tO = tmem + lane_off + C::COL_O + t * D;
-    const int row_limit = CAUSAL ? min(p.Nkv, row + off + 1) : p.Nkv;
     const float sl2 = p.scale_log2;
-    float m = -INFINITY, l = 0.f;
+    int g = 0, local = 0;
     bool ok = true;
-
-    for (int j = 0; j < n; ++j) {
-      ok = warp_wait(&bars->s_full[t], j & 1, p.wait_ns, abort_flag, 30 + t);
-      if (!ok) break;
-      tc_fence_after();
-      uint32_t sr[C::BN];
+    for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++local) {
+      const int qt = item_qt(it), bh = item_bh(it);
+      const int n = item_ntiles(qt);
+      const int row = qt * 2 * C::BM + t * C::BM + r;
+      const int row_limit = CAUSAL ? min(p.Nkv, row + off + 1) : p.Nkv;
+      float m = -INFINITY, l = 0.f;
+      // a warp whose rows are all padding (past Nq) skips the arithmetic: its P rows
+      // only feed output rows that are never stored
+      const bool idle = __all_sync(0xffffffffu, row >= p.Nq);
+      for (int j = 0; j < n; ++j, ++g) {
+        ok = warp_wait(&bars->s_full[t], g & 1, p.wait_ns, abort_flag, 30 + t);
+        if (!ok) break;
+        if (!idle) {
+          tc_fence_after();
+          uint32_t sr[C::BN];
 #pragma unroll
-      for (int c = 0; c < C::BN / 32; ++c) tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
-      tmem_wait_ld();
-      float f[C::BN];
-      const int lim = row_limit - j * C::BN;
-#pragma unroll
-      for (int c = 0; c < C::BN; ++c) f[c] = __uint_as_float(sr[c]);
-      if (lim < C::BN) {
-#pragma unroll
-        for (int c = 0; c < C::BN; ++c) f[c] = (c < lim) ? f[c] : -INFINITY;
-      }
-      float mx = f[0];
-#pragma unroll
-      for (int c = 1; c < C::BN; ++c) mx = fmaxf(mx, f[c]);
-      const float m_new = fmaxf(m, mx * sl2);
-      const float base = (m_new == -INFINITY) ? 0.f : m_new;
-      const float alpha = (m_new == m) ? 1.f : ex2(m - base);
-      float rs = 0.f;
-#pragma unroll
-      for (int c = 0; c < C::BN / 32; ++c) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float p0 = ex2(fmaf(f[c * 32 + 2 * i], sl2, -base));
-          const float p1 = ex2(fmaf(f[c * 32 + 2 * i + 1], sl2, -base));
-          rs += p0 + p1;
-          pk[i] = pack_bf16x2(p0, p1);
-        }
-        tmem_st16(tS + c * 16, pk);
-      }
-      l = l * alpha + rs;
-      // u (TMEM) holds the P.V sums of tiles < j; rescale its rows whose max rose
-      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(tO + c * 32, o);
+          for (int c = 0; c < C::BN / 32; ++c)
+            tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
           tmem_wait_ld();
+          float f[C::BN];
+          const int lim = row_limit - j * C::BN;  // columns >= lim are masked for this row
+          const bool masked = __any_sync(0xffffffffu, lim < C::BN);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32(tO + c * 32, o);
+          for (int c = 0; c < C::BN; ++c) f[c] = __uint_as_float(sr[c]);
+          if (masked) {
+#pragma unroll
+            for (int c = 0; c < C::BN; ++c) f[c] = (c < lim) ? f[c] : -INFINITY;
+          }
+          float mx8[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) mx8[k] = f[k];
+#pragma unroll
+          for (int c = 8; c < C::BN; c += 8)
+#pragma unroll
+            for (int k = 0; k < 8; ++k) mx8[k] = fmaxf(mx8[k], f[c + k]);
+          const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                 fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+          const float m_new = fmaxf(m, mx * sl2);
+          const float base = (m_new == -INFINITY) ? 0.f : m_new;
+          const float alpha = (m_new == m) ? 1.f : ex2(m - base);
+          const float2 sl2v = make_float2(sl2, sl2), nbase = make_float2(-base, -base);
+          float2 rs2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                           make_float2(0.f, 0.f)};
+          if (masked) {
+            // boundary tile: every exponential on the SFU (exactly 0 for masked scores);
+            // 32-column chunks that are masked for the whole warp are skipped
+#pragma unroll
+            for (int c = 0; c < C::BN / 32; ++c) {
+              uint32_t pk[16];
+              if (__all_sync(0xffffffffu, lim <= c * 32)) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) pk[i] = 0u;
+              } else {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                  const float2 x =
+                      __ffma2_rn(make_float2(f[c * 32 + 2 * i], f[c * 32 + 2 * i + 1]), sl2v, nbase);
+                  const float2 pv = make_float2(ex2(x.x), ex2(x.y));
+                  rs2[i & 3] = __fadd2_rn(rs2[i & 3], pv);
+                  pk[i] = pack_bf16x2(pv.x, pv.y);
+                }
+              }
+              tmem_st16(tS + c * 16, pk);
+            }
+          } else {
+            // interior tile: pairs FWD_EMU_PAIRS of every 8 take the FMA-pipe exponential
+#pragma unroll
+            for (int c = 0; c < C::BN / 32; ++c) {
+              uint32_t pk[16];
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const float2 x = __ffma2_rn(make_float2(f[c * 32 + 2 * i], f[c * 32 + 2 * i + 1]), sl2v, nbase);
+                const float2 pv = ((FWD_EMU_PAIRS >> (i & 7)) & 1) ? exp2_fma2(x) : make_float2(ex2(x.x), ex2(x.y));
+                rs2[i & 3] = __fadd2_rn(rs2[i & 3], pv);
+                pk[i] = pack_bf16x2(pv.x, pv.y);
+              }
+              tmem_st16(tS + c * 16, pk);
+            }
+          }
+          const float2 rsa = __fadd2_rn(__fadd2_rn(rs2[0], rs2[1]), __fadd2_rn(rs2[2], rs2[3]));
+          l = l * alpha + (rsa.x + rsa.y);
+          // u (TMEM) holds the P.V sums of tiles < j; rescale its rows whose max rose
+          if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t o[32];
+              tmem_ld32(tO + c * 32, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 32; i += 2) {
+                const float2 v = __fmul2_rn(make_float2(__uint_as_float(o[i]), __uint_as_float(o[i + 1])),
+                                            make_float2(alpha, alpha));
+                o[i] = __float_as_uint(v.x);
+                o[i + 1] = __float_as_uint(v.y);
+              }
+              tmem_st32(tO + c * 32, o);
+            }
+          }
+          tmem_wait_st();
+          m = m_new;
         }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->p_full[t]);
       }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->p_full[t]);
-      m = m_new;
-    }
-    if (ok) ok = warp_wait(&bars->o_final[t], 0, p.wait_ns, abort_flag, 40 + t);
-    if (ok) {
+      if (ok) ok = warp_wait(&bars->o_final[t], local & 1, p.wait_ns, abort_flag, 40 + t);
+      if (!ok) break;
+      if (idle) continue;
       tc_fence_after();
       const float inv = 1.f / l;
       __nv_bfloat16* orow = p.o + (size_t(bh) * p.Nq + row) * D;

@@ -183,6 +183,14 @@ void fa_set_wait_limit_ns(uint64_t ns);
  */
 fa_status fa_selftest_wait_timeout(void* stream);
 
+/*
+ * fa_selftest_exp2 — evaluates, for n device floats x (x <= 0), the FMA-pipe 2^x that the
+ * forward kernel uses for part of each unmasked score tile (range reduction plus a
+ * fitted degree-4 polynomial, relative error <= 2.7e-6 for x in [-126, 0]), writing y.
+ * For tests of that approximation against exp2.
+ */
+fa_status fa_selftest_exp2(const float* x, float* y, int n, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -147,3 +147,20 @@ def test_wait_timeout_sets_status_without_fault():
     # the context is still usable
     x = torch.ones(4, device="cuda")
     assert x.sum().item() == 4.0
+
+
+def test_fma_pipe_exp2_against_exp2():
+    """The FMA-pipe 2^x used for part of each unmasked tile stays within 3e-6 of exp2."""
+    import ctypes
+
+    x = torch.cat([torch.linspace(-126.0, 0.0, 1 << 20, dtype=torch.float64),
+                   -torch.rand(1 << 20, dtype=torch.float64, generator=torch.Generator().manual_seed(5)) * 30])
+    xf = x.float().cuda()
+    y = torch.empty_like(xf)
+    st = fa.lib().fa_selftest_exp2(ctypes.c_void_p(xf.data_ptr()), ctypes.c_void_p(y.data_ptr()), xf.numel(),
+                                   ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == 0
+    torch.cuda.synchronize()
+    ref = torch.exp2(xf.double().cpu())
+    rel = ((y.double().cpu() - ref).abs() / ref).max().item()
+    assert rel <= 3e-6, rel
