@@ -16,13 +16,12 @@
 // ("No basta con promediar los resultados de los bloques": block results are never
 // simply averaged).  A request that fits in one split writes its output directly.
 //
-// Data path: the step is bound by reading K and V from device memory.  Every thread
-// copies its own 16-byte pieces of each 4 KB (block, kv head) slab into shared memory
-// with cp.async (a ring of STAGES blocks per warp) and later reads back exactly those
-// pieces, so no intra-warp synchronisation is needed and the reads are
-// conflict-free.  The pieces are chosen so that they already form mma.sync fragments:
-// the head dimension is permuted consistently between q and K (a dot product does not
-// depend on the order of its terms) and between V and the output columns.
+// Data path: the step is bound by reading K and V from device memory.  Each warp owns
+// a ring of STAGES shared-memory stages; its lane 0 prefetches the warp's block-table
+// entries once, then issues TMA loads of each 4 KB (block, kv head) slab (two 64-column
+// boxes with the 128-byte swizzle, so ldmatrix reads are conflict-free) addressed by the
+// physical block id.  Scores and P.V use mma.sync m16n8k16 with the group's query heads
+// as the 16 rows (rows >= G are zero): ldmatrix for K, ldmatrix.trans for V.
 #pragma once
 #include "common.cuh"
 
@@ -34,14 +33,16 @@ constexpr int WARPS = 4;
 constexpr int STAGES = 3;       // blocks in flight per warp
 constexpr int CHUNK = 32;       // logical blocks per CTA (split size = 512 tokens)
 constexpr int SLAB = BS * D * 2;  // 4096 bytes: one (block, kv head) slab of K or V
-constexpr int SMEM = WARPS * STAGES * 2 * SLAB;
+constexpr int STAGE_BYTES = 2 * SLAB;
+constexpr int OFF_BAR = WARPS * STAGES * STAGE_BYTES;
+constexpr int SMEM = OFF_BAR + WARPS * STAGES * 8 + 1024;
 constexpr int MAX_G = 16;
+constexpr int OP = D + 8;  // padded row of the warp-merge buffer (floats)
+static_assert(WARPS * MAX_G * OP * 4 + 2 * WARPS * MAX_G * 4 <= OFF_BAR, "merge buffer must fit the stages");
 }  // namespace dec
 
 struct DecodeParams {
   const __nv_bfloat16* q;
-  const __nv_bfloat16* kc;
-  const __nv_bfloat16* vc;
   const int* bt;
   const int* ctx;
   __nv_bfloat16* o;
@@ -50,16 +51,8 @@ struct DecodeParams {
   float* part_lse;
   int R, Hq, Hkv, max_blocks, num_blocks, max_splits;
   float scale_log2;
+  uint64_t wait_ns;
 };
-
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
 
 __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -69,9 +62,39 @@ __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-__global__ void __launch_bounds__(dec::WARPS * 32) fa_paged_decode_kernel(const DecodeParams p) {
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t smem_dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
+      "[%2];" ::"r"(smem_dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+
+// Byte offset of 16-byte chunk `chunk` (0..15) of slab row `row` (0..15) in a stage
+// half-pair: chunks 0-7 live in the first 2 KB box, 8-15 in the second, each row 128 B
+// with the 128-byte swizzle (chunk index XOR row % 8).
+__device__ __forceinline__ uint32_t slab_off(int row, int chunk) {
+  return uint32_t((chunk >> 3) * 2048 + row * 128 + (((chunk & 7) ^ (row & 7)) << 4));
+}
+
+__global__ void __launch_bounds__(dec::WARPS * 32)
+    fa_paged_decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                           const DecodeParams p) {
   using namespace dec;
-  extern __shared__ __align__(16) uint8_t dsmem[];
+  extern __shared__ uint8_t dsmem_raw[];
+  uint8_t* dsmem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) & ~uintptr_t(1023));
   const int s = blockIdx.x, g = blockIdx.y, r = blockIdx.z;
   const int G = p.Hq / p.Hkv;
   const int ctx = p.ctx[r];
@@ -86,64 +109,58 @@ __global__ void __launch_bounds__(dec::WARPS * 32) fa_paged_decode_kernel(const 
   const int b1 = min(nblk, b0 + CHUNK);
 
   const int warp = warp_id(), lane = lane_id();
-  const int gq = lane >> 2;  // mma group id: query head row (and +8), key token, output column group
+  const int gq = lane >> 2;  // mma group id: query-head row, key token, output column
   const int t4 = lane & 3;
-  const int nb = (b1 - b0 - warp + WARPS - 1) / WARPS;  // blocks for this warp (may be <= 0)
+  const int nb = max(0, (b1 - b0 - warp + WARPS - 1) / WARPS);  // this warp's blocks
+  uint64_t* bars = reinterpret_cast<uint64_t*>(dsmem + OFF_BAR) + warp * STAGES;
+  const uint32_t sbase = smem_u32(dsmem) + warp * STAGES * STAGE_BYTES;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) abort_flag = 0;
+  if (lane == 0)
+    for (int st = 0; st < STAGES; ++st) mbar_init(&bars[st], 1);
+  fence_barrier_init();
+  __syncthreads();
 
-  // q fragments (A operand, 16 rows = heads of the group, zero past G), with the head
-  // dimension permuted: virtual k (2*t4 + {0,1}, 2*t4 + 8 + {0,1}) of k-step ks is
-  // physical d = 32*t4 + 4*ks + {0,1} and {2,3}.
+  // physical block of this warp's i-th block, held by lane i (CHUNK / WARPS <= 32)
+  int my_phys = 0;
+  if (lane < nb) {
+    my_phys = p.bt[size_t(r) * p.max_blocks + b0 + warp + lane * WARPS];
+    if (my_phys < 0 || my_phys >= p.num_blocks) {
+      set_status(FA_ERR_INVALID_ARG, 101);
+      my_phys = 0;  // never address an out-of-range block; the result is flagged invalid
+    }
+  }
+  // the whole warp calls issue(i) (the shuffle needs every lane); lane 0 issues the loads
+  auto issue = [&](int i) {
+    const int phys = __shfl_sync(0xffffffffu, my_phys, i);
+    if (lane == 0) {
+      const int row = (phys * p.Hkv + g) * BS;
+      uint64_t* bar = &bars[i % STAGES];
+      const uint32_t st = sbase + (i % STAGES) * STAGE_BYTES;
+      mbar_arrive_expect_tx(bar, STAGE_BYTES);
+      tma_load_2d(st, &tmK, bar, 0, row);
+      tma_load_2d(st + 2048, &tmK, bar, 64, row);
+      tma_load_2d(st + SLAB, &tmV, bar, 0, row);
+      tma_load_2d(st + SLAB + 2048, &tmV, bar, 64, row);
+    }
+  };
+  for (int i = 0; i < min(nb, STAGES); ++i) issue(i);
+
+  // q fragments (A operand): rows = heads of the group (zero past G), natural d order
   uint32_t qa[8][4];
   {
     const int h0 = g * G + gq, h1 = g * G + gq + 8;
-    const uint32_t* q0 = reinterpret_cast<const uint32_t*>(p.q + (size_t(r) * p.Hq + h0) * D + 32 * t4);
-    const uint32_t* q1 = reinterpret_cast<const uint32_t*>(p.q + (size_t(r) * p.Hq + h1) * D + 32 * t4);
     const bool v0 = gq < G, v1 = gq + 8 < G;
+    const uint32_t* q0 = reinterpret_cast<const uint32_t*>(p.q + (size_t(r) * p.Hq + (v0 ? h0 : 0)) * D);
+    const uint32_t* q1 = reinterpret_cast<const uint32_t*>(p.q + (size_t(r) * p.Hq + (v1 ? h1 : 0)) * D);
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
-      qa[ks][0] = v0 ? q0[2 * ks] : 0u;
-      qa[ks][1] = v1 ? q1[2 * ks] : 0u;
-      qa[ks][2] = v0 ? q0[2 * ks + 1] : 0u;
-      qa[ks][3] = v1 ? q1[2 * ks + 1] : 0u;
+      qa[ks][0] = v0 ? q0[8 * ks + t4] : 0u;
+      qa[ks][1] = v1 ? q1[8 * ks + t4] : 0u;
+      qa[ks][2] = v0 ? q0[8 * ks + 4 + t4] : 0u;
+      qa[ks][3] = v1 ? q1[8 * ks + 4 + t4] : 0u;
     }
   }
-
-  const uint32_t sbase = smem_u32(dsmem) + warp * STAGES * 2 * SLAB;
-  const size_t slab_elems = size_t(BS) * D;
-  const int* bt_row = p.bt + size_t(r) * p.max_blocks;
-
-  // Issue the copies of this warp's i-th block into stage i % STAGES (always commits a
-  // group, possibly empty, so group counting stays uniform).
-  auto issue = [&](int i) {
-    if (i < nb) {
-      const int lb = b0 + warp + i * WARPS;
-      int phys = bt_row[lb];
-      if (phys < 0 || phys >= p.num_blocks) {
-        set_status(FA_ERR_INVALID_ARG, 101);
-        phys = 0;  // never dereference an out-of-range id; the result is flagged invalid
-      }
-      const __nv_bfloat16* ks = p.kc + (size_t(phys) * p.Hkv + g) * slab_elems;
-      const __nv_bfloat16* vs = p.vc + (size_t(phys) * p.Hkv + g) * slab_elems;
-      const uint32_t dk = sbase + (i % STAGES) * 2 * SLAB;
-      const uint32_t dv = dk + SLAB;
-      // K: tokens gq and gq + 8, d in [32*t4, 32*t4 + 32): 4 pieces each
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const int tok = gq + 8 * (c >> 2);
-        cp_async16(dk + (c * 32 + lane) * 16, ks + tok * D + 32 * t4 + 8 * (c & 3));
-      }
-      // V: tokens 2*t4 + {0, 1, 8, 9}, d in [16*gq, 16*gq + 16): 2 pieces each
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const int tok = 2 * t4 + (c >> 1 & 1) + 8 * (c >> 2);
-        cp_async16(dv + (c * 32 + lane) * 16, vs + tok * D + 16 * gq + 8 * (c & 1));
-      }
-    }
-    cp_async_commit();
-  };
-
-#pragma unroll
-  for (int i = 0; i < STAGES; ++i) issue(i);
 
   float m0 = -INFINITY, m1 = -INFINITY;  // running max (log2 units) of rows gq, gq + 8
   float l0 = 0.f, l1 = 0.f;              // this thread's share of the running sums
@@ -151,29 +168,28 @@ __global__ void __launch_bounds__(dec::WARPS * 32) fa_paged_decode_kernel(const 
 #pragma unroll
   for (int nt = 0; nt < 16; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
   const float sl2 = p.scale_log2;
+  // ldmatrix row addresses: lane -> (matrix mi = lane / 8, row rr = lane % 8)
+  const int mi = lane >> 3, rr = lane & 7;
+  const int k_tok = rr + 8 * (mi >> 1), k_chunk_lo = mi & 1;  // K: (token, d-chunk parity)
+  const int v_tok = rr + 8 * (mi & 1), v_chunk_hi = mi >> 1;  // V: (token, n-tile parity)
 
-  for (int i = 0; i < nb; ++i) {
-    cp_async_wait<STAGES - 1>();
-    const uint32_t dk = sbase + (i % STAGES) * 2 * SLAB;
-    const uint32_t dv = dk + SLAB;
+  bool ok = true;
+  for (int i = 0; i < nb && ok; ++i) {
+    ok = warp_wait(&bars[i % STAGES], (i / STAGES) & 1, p.wait_ns, &abort_flag, 102);
+    if (!ok) break;
+    const uint32_t sk = sbase + (i % STAGES) * STAGE_BYTES;
+    const uint32_t sv = sk + SLAB;
     const int lb = b0 + warp + i * WARPS;
     const int valid = min(BS, ctx - lb * BS);  // tokens of this block that are cached
 
-    // ---- scores S[head][token] = q . k over the permuted head dimension
+    // ---- scores S[head][token] = q . k
     float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-      uint32_t kr[16];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint4 v4;
-        asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
-                     : "=r"(v4.x), "=r"(v4.y), "=r"(v4.z), "=r"(v4.w)
-                     : "r"(dk + ((nt * 4 + c) * 32 + lane) * 16));
-        kr[4 * c] = v4.x; kr[4 * c + 1] = v4.y; kr[4 * c + 2] = v4.z; kr[4 * c + 3] = v4.w;
-      }
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks) mma_bf16_16816(sc[nt], qa[ks], kr[2 * ks], kr[2 * ks + 1]);
+    for (int ks = 0; ks < 8; ++ks) {
+      uint32_t b00, b01, b10, b11;
+      ldsm_x4(sk + slab_off(k_tok, 2 * ks + k_chunk_lo), b00, b01, b10, b11);
+      mma_bf16_16816(sc[0], qa[ks], b00, b01);
+      mma_bf16_16816(sc[1], qa[ks], b10, b11);
     }
     // ---- mask tokens past ctx (selection, so garbage in unused slots cannot leak)
     if (valid < BS) {
@@ -189,7 +205,7 @@ __global__ void __launch_bounds__(dec::WARPS * 32) fa_paged_decode_kernel(const 
     mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
     mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
     mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-    const float n0 = fmaxf(m0, mx0 * sl2), n1 = fmaxf(m1, mx1 * sl2);  // the first block has a valid token
+    const float n0 = fmaxf(m0, mx0 * sl2), n1 = fmaxf(m1, mx1 * sl2);  // every block has a cached token
     const float a0 = ex2(m0 - n0), a1 = ex2(m1 - n1);                  // 0 on the first block
     m0 = n0;
     m1 = n1;
@@ -216,57 +232,42 @@ __global__ void __launch_bounds__(dec::WARPS * 32) fa_paged_decode_kernel(const 
     pa[2] = pack_bf16x2(pr[1][0], pr[1][1]);
     pa[3] = pack_bf16x2(pr[1][2], pr[1][3]);
 
-    // ---- u += P V: V pieces -> B fragments (two tokens per 32-bit register)
-    uint32_t vr[4][4];  // [token slot: 2t4, 2t4+1, 2t4+8, 2t4+9][4 x bf16x2 of 8 d's] per half
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-#pragma unroll
-      for (int ts = 0; ts < 4; ++ts) {
-        const int c = 2 * ts + half;  // piece: token slot ts, d half
-        asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
-                     : "=r"(vr[ts][0]), "=r"(vr[ts][1]), "=r"(vr[ts][2]), "=r"(vr[ts][3])
-                     : "r"(dv + (c * 32 + lane) * 16));
-      }
-      if (valid < BS) {  // zero V rows of uncached tokens (P is 0 there; 0 * NaN would not be)
-#pragma unroll
-        for (int ts = 0; ts < 4; ++ts) {
-          const int tok = 2 * t4 + (ts & 1) + 8 * (ts >> 1);
-          if (tok >= valid) vr[ts][0] = vr[ts][1] = vr[ts][2] = vr[ts][3] = 0u;
-        }
-      }
-      // output column n-tile nt holds physical d = 16*n + nt; this half covers nt in [8*half, 8*half+8)
-#pragma unroll
-      for (int w = 0; w < 4; ++w) {
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int nt = 8 * half + 2 * w + e;
-          const uint32_t sel = e ? 0x7632u : 0x5410u;
-          const uint32_t bb0 = __byte_perm(vr[0][w], vr[1][w], sel);
-          const uint32_t bb1 = __byte_perm(vr[2][w], vr[3][w], sel);
-          mma_bf16_16816(acc[nt], pa, bb0, bb1);
-        }
-      }
+    // ---- u += P V; this thread's B fragments hold tokens 2t4, 2t4+1 (b0), +8 (b1)
+    uint32_t keep0 = 0xffffffffu, keep1 = 0xffffffffu;
+    if (valid < BS) {  // zero V of uncached tokens (P is 0 there; 0 * NaN would not be)
+      keep0 = (2 * t4 < valid ? 0x0000ffffu : 0u) | (2 * t4 + 1 < valid ? 0xffff0000u : 0u);
+      keep1 = (2 * t4 + 8 < valid ? 0x0000ffffu : 0u) | (2 * t4 + 9 < valid ? 0xffff0000u : 0u);
     }
-    issue(i + STAGES);
+#pragma unroll
+    for (int nt = 0; nt < 16; nt += 2) {
+      uint32_t v00, v01, v10, v11;
+      ldsm_x4_t(sv + slab_off(v_tok, nt + v_chunk_hi), v00, v01, v10, v11);
+      mma_bf16_16816(acc[nt], pa, v00 & keep0, v01 & keep1);
+      mma_bf16_16816(acc[nt + 1], pa, v10 & keep0, v11 & keep1);
+    }
+    // all lanes have read this stage: refill it
+    __syncwarp();
+    if (i + STAGES < nb) {
+      fence_proxy_async_smem();
+      issue(i + STAGES);
+    }
   }
-  cp_async_wait<0>();
 
-  // ---- merge the 4 warps' (m, l, u) states
+  // ---- merge the warps' (m, l, u) states
   l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
   l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
   l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
   l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
   __syncthreads();  // all warps done with their stages: reuse shared memory
-  float* so = reinterpret_cast<float*>(dsmem);              // [WARPS][MAX_G][D]
-  float* sm = so + WARPS * MAX_G * D;                        // [WARPS][MAX_G]
-  float* sl = sm + WARPS * MAX_G;                            // [WARPS][MAX_G]
+  if (abort_flag) return;
+  float* so = reinterpret_cast<float*>(dsmem);  // [WARPS][MAX_G][OP]
+  float* sm = so + WARPS * MAX_G * OP;          // [WARPS][MAX_G]
+  float* sl = sm + WARPS * MAX_G;               // [WARPS][MAX_G]
 #pragma unroll
   for (int nt = 0; nt < 16; ++nt) {
-    const int d0 = 16 * (2 * t4) + nt, d1 = 16 * (2 * t4 + 1) + nt;
-    so[(warp * MAX_G + gq) * D + d0] = acc[nt][0];
-    so[(warp * MAX_G + gq) * D + d1] = acc[nt][1];
-    so[(warp * MAX_G + gq + 8) * D + d0] = acc[nt][2];
-    so[(warp * MAX_G + gq + 8) * D + d1] = acc[nt][3];
+    const int d0 = 8 * nt + 2 * t4;
+    *reinterpret_cast<float2*>(&so[(warp * MAX_G + gq) * OP + d0]) = make_float2(acc[nt][0], acc[nt][1]);
+    *reinterpret_cast<float2*>(&so[(warp * MAX_G + gq + 8) * OP + d0]) = make_float2(acc[nt][2], acc[nt][3]);
   }
   if (t4 == 0) {
     sm[warp * MAX_G + gq] = m0;
@@ -287,7 +288,7 @@ __global__ void __launch_bounds__(dec::WARPS * 32) fa_paged_decode_kernel(const 
       const float mw = sm[w * MAX_G + hr];
       const float wt = (mw == -INFINITY) ? 0.f : ex2(mw - M);
       L += sl[w * MAX_G + hr] * wt;
-      U += so[(w * MAX_G + hr) * D + d] * wt;
+      U += so[(w * MAX_G + hr) * OP + d] * wt;
     }
     const int h = g * G + hr;
     const float lse_nat = (M + __log2f(L)) * 0.69314718055994531f;

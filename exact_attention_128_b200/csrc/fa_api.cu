@@ -51,6 +51,20 @@ bool make_map_bf16(CUtensorMap* m, const void* base, int d, int rows, int planes
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D bf16 map over a paged cache viewed as [rows][128] with a (64, 16) box and the
+// 128-byte swizzle: one box is half of one (block, kv head) slab.
+bool make_map_cache(CUtensorMap* m, const void* base, long rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {128, cuuint64_t(rows)};
+  cuuint64_t strides[1] = {256};
+  cuuint32_t box[2] = {64, 16};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <typename K>
 cudaError_t set_smem(K kernel, int bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
@@ -301,13 +315,15 @@ fa_status fa_paged_decode(const void* q, const void* k_cache, const void* v_cach
   float* part_o = static_cast<float*>(workspace);
   float* part_lse =
       reinterpret_cast<float*>(static_cast<char*>(workspace) + align256(size_t(R) * Hq * max_splits * d * 4));
-  DecodeParams prm{static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k_cache),
-                   static_cast<const __nv_bfloat16*>(v_cache), block_table, ctx_lens,
-                   static_cast<__nv_bfloat16*>(o), lse, part_o, part_lse, R, Hq, Hkv, max_blocks_per_seq,
-                   num_blocks, max_splits, scale * 1.4426950408889634f};
+  DecodeParams prm{static_cast<const __nv_bfloat16*>(q), block_table, ctx_lens, static_cast<__nv_bfloat16*>(o),
+                   lse, part_o, part_lse, R, Hq, Hkv, max_blocks_per_seq, num_blocks, max_splits,
+                   scale * 1.4426950408889634f, g_wait_ns};
+  CUtensorMap mk, mv;
+  const long cache_rows = long(num_blocks) * Hkv * dec::BS;
+  if (!make_map_cache(&mk, k_cache, cache_rows) || !make_map_cache(&mv, v_cache, cache_rows)) return FA_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (set_smem(fa_paged_decode_kernel, dec::SMEM) != cudaSuccess) return FA_ERR_CUDA;
-  fa_paged_decode_kernel<<<dim3(max_splits, Hkv, R), dec::WARPS * 32, dec::SMEM, st>>>(prm);
+  fa_paged_decode_kernel<<<dim3(max_splits, Hkv, R), dec::WARPS * 32, dec::SMEM, st>>>(mk, mv, prm);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   fa_paged_decode_combine_kernel<<<R * Hq, dec::D, 0, st>>>(prm);
   return launched();
