@@ -14,16 +14,18 @@
 //      +inf, so padded rows get P = 0), and zeroes the fp32 dQ accumulator.
 //   2. fa_bwd_bf16_kernel: one CTA per (128-key tile j, batch, key/value head).  It keeps
 //      K_j, V_j in shared memory and walks the G query heads of its group and their
-//      query tiles i (causal: only tiles at or below the diagonal):
+//      query tiles i (causal: only tiles at or below the diagonal).  Each step is split
+//      into query halves A (rows 0-63) and B (64-127) so the softmax-gradient of one half
+//      overlaps the tensor-core work of the other:
 //        warp 0      TMA producer: K_j, V_j once; Q_i, dO_i, lse_i, D_i per step (2 stages)
-//        warp 1      MMA issuer (one thread): S^T = K_j Q_i^T and dP^T = V_j dO_i^T into
-//                    TMEM; then dV += P^T dO_i and dK += dS^T Q_i with P^T, dS^T read from
-//                    TMEM, and dQ_i = dS K_j with dS read from shared memory.
-//        warps 4-7   one thread per key (TMEM lane): P^T and dS^T from S^T, dP^T, lse, D;
-//                    P^T and dS^T (bf16) go back over S^T and dP^T in TMEM, dS^T also to
-//                    shared memory (swizzled, query-major) for the dQ MMA.  At the end
-//                    they write dK_j and dV_j.
-//        warps 8-11  one thread per query row: read dQ_i from TMEM and add it into the fp32
+//        warp 1      MMA issuer (one thread): per half, S^T = K_j Q_h^T and dP^T = V_j dO_h^T
+//                    into TMEM; per half, dV += P^T dO_h and dK += dS^T Q_h with P^T, dS^T
+//                    read from TMEM; then dQ_i = dS K_j with dS read from shared memory.
+//        warps 4-7   half A, warps 8-11 half B; one thread per key (TMEM lane): P^T and
+//                    dS^T from S^T, dP^T, lse, D; P^T and dS^T (bf16) go back over S^T and
+//                    dP^T in TMEM, dS^T also to shared memory (swizzled, query-major) for
+//                    the dQ MMA.  At the end half A's warps write dK_j, half B's dV_j.
+//        warps 12-15 one thread per query row: read dQ_i from TMEM and add it into the fp32
 //                    accumulator with vector reductions (red.global.add.v4.f32).
 //   3. fa_bwd_finalize_kernel: fp32 dQ accumulator -> bf16 dq (only for bf16 gradients;
 //      fp32 gradients accumulate straight into dq).
@@ -47,14 +49,18 @@ struct BwdCfg {
   static constexpr int OFF_V = OFF_K + TILE;
   static constexpr int OFF_Q = OFF_V + TILE;           // + stage * TILE
   static constexpr int OFF_DO = OFF_Q + 2 * TILE;      // + stage * TILE
-  static constexpr int OFF_DS = OFF_DO + 2 * TILE;     // [2 query chunks][128 keys][128 B]
-  static constexpr int OFF_STAT = OFF_DS + 128 * 128 * 2;  // per stage: lse2[128], D[128]
+  // d = 64 issues the next step's half-A scores before the current step's dQ MMA, so
+  // the dS tile that dQ reads is double-buffered; d = 128 has no room and keeps one.
+  static constexpr bool EARLY = (D == 64);
+  static constexpr int DS_BUF = EARLY ? 2 : 1;
+  static constexpr int OFF_DS = OFF_DO + 2 * TILE;     // DS_BUF x [2 query chunks][128 keys][128 B]
+  static constexpr int OFF_STAT = OFF_DS + DS_BUF * 128 * 128 * 2;  // per stage: lse2[128], D[128]
   static constexpr int OFF_BAR = OFF_STAT + 2 * 2 * 512;
   // D = 128 fills the 227 KB limit exactly, leaving no room to re-align the base: that
   // variant relies on the dynamic shared memory starting 1024-byte aligned and checks it.
   static constexpr int SLACK = (D == 128) ? 0 : 1024;
   static constexpr int SMEM = OFF_BAR + 256 + SLACK;
-  static constexpr int THREADS = 384;
+  static constexpr int THREADS = 512;
   static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DV = 256, COL_DK = 256 + D;
   static constexpr int NQB = (D == 64) ? 2 : 1;  // dQ TMEM buffers
   __host__ __device__ static constexpr uint32_t col_dq(int buf) { return D == 64 ? uint32_t(384 + 64 * buf) : COL_DP; }
@@ -77,8 +83,8 @@ struct BwdBars {
   uint64_t kv_full;
   uint64_t qdo_full[2];
   uint64_t qdo_empty[2];
-  uint64_t sdp_full;
-  uint64_t ds_ready;
+  uint64_t sdp_full[2];  // per query half
+  uint64_t ds_ready[2];  // per query half
   uint64_t dq_full[2];
   uint64_t dq_free[2];
   uint64_t dkdv_full;
@@ -158,7 +164,7 @@ __global__ void __launch_bounds__(256) fa_bwd_finalize_kernel(const float* acc, 
 
 // ------------------------------------------------------------------------------ 2
 template <int D, bool CAUSAL>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(512, 1)
     fa_bwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                        const BwdParams p) {
@@ -193,9 +199,9 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(&bars->qdo_empty[s], 1);
       mbar_init(&bars->dq_full[s], 1);
       mbar_init(&bars->dq_free[s], 4);
+      mbar_init(&bars->sdp_full[s], 1);
+      mbar_init(&bars->ds_ready[s], 4);
     }
-    mbar_init(&bars->sdp_full, 1);
-    mbar_init(&bars->ds_ready, 4);
     mbar_init(&bars->dkdv_full, 1);
     bars->abort_flag = 0;
     fence_barrier_init();
@@ -242,113 +248,171 @@ __global__ void __launch_bounds__(384, 1)
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
+    // Each step is split into query halves A (rows 0-63) and B (64-127): S^T and dP^T of
+    // half B run on the tensor core while half A's softmax-gradient is computed, and
+    // half A's dV/dK MMAs run while half B's is.
     if (lane == 0 && n_steps > 0) {
-      constexpr uint32_t idKK = idesc_bf16_f32(128, 128, 0);  // S^T, dP^T: both operands K-major
-      constexpr uint32_t idTS = idesc_bf16_f32(128, D, 1);    // dV, dK: B (dO, Q) MN-major
-      constexpr uint32_t idQ = idesc_bf16_f32(128, D, 1) | (1u << 15);  // dQ: A (dS) and B (K) MN-major
-      bool ok = mbar_wait(&bars->kv_full, 0, p.wait_ns, abort_flag, 210);
-      for (int s = 0; s < n_steps && ok; ++s) {
+      constexpr uint32_t idKK = idesc_bf16_f32(128, 64, 0);             // S^T, dP^T halves: N = 64
+      constexpr uint32_t idTS = idesc_bf16_f32(128, D, 1);              // dV, dK: B (dO, Q) MN-major
+      constexpr uint32_t idQ = idesc_bf16_f32(128, D, 1) | (1u << 15);  // dQ: A (dS), B (K) MN-major
+      // S^T and dP^T of query half hf of step s (commit sdp_full[hf])
+      auto issue_sdp = [&](int s, int hf) {
         const int st = s & 1;
-        ok = mbar_wait(&bars->qdo_full[st], (s >> 1) & 1, p.wait_ns, abort_flag, 211);
-        if (!ok) break;
-        if constexpr (D == 128) {  // dP^T overwrites the previous dQ: wait for its drain
-          if (s > 0 && !(ok = mbar_wait(&bars->dq_free[0], (s - 1) & 1, p.wait_ns, abort_flag, 212))) break;
+        const uint32_t sQ = sbase + C::OFF_Q + st * C::TILE, sO = sbase + C::OFF_DO + st * C::TILE;
+        // rows [64*hf, 64*hf + 64) of Q and dO: 64 rows * 128 B further in each block
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint32_t koff = (ks >> 2) * 128 * 128 + (ks & 3) * 32;
+          mma_ss(tmem + C::COL_S + 64 * hf, sdesc_sw128(sbase + C::OFF_K + koff, 16, 1024),
+                 sdesc_sw128(sQ + koff + hf * 64 * 128, 16, 1024), idKK, ks > 0);
         }
-        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint32_t koff = (ks >> 2) * 128 * 128 + (ks & 3) * 32;
+          mma_ss(tmem + C::COL_DP + 64 * hf, sdesc_sw128(sbase + C::OFF_V + koff, 16, 1024),
+                 sdesc_sw128(sO + koff + hf * 64 * 128, 16, 1024), idKK, ks > 0);
+        }
+        mma_commit(&bars->sdp_full[hf]);
+      };
+      // dV += P^T dO ; dK += dS^T Q for query half hf of step s (K dimension = 64 queries)
+      auto issue_dvdk = [&](int s, int hf) {
+        const int st = s & 1;
         const uint32_t sQ = sbase + C::OFF_Q + st * C::TILE, sO = sbase + C::OFF_DO + st * C::TILE;
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-          const uint32_t koff = (ks >> 2) * 128 * 128 + (ks & 3) * 32;
-          mma_ss(tmem + C::COL_S, sdesc_sw128(sbase + C::OFF_K + koff, 16, 1024), sdesc_sw128(sQ + koff, 16, 1024),
-                 idKK, ks > 0);
-        }
-#pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-          const uint32_t koff = (ks >> 2) * 128 * 128 + (ks & 3) * 32;
-          mma_ss(tmem + C::COL_DP, sdesc_sw128(sbase + C::OFF_V + koff, 16, 1024), sdesc_sw128(sO + koff, 16, 1024),
-                 idKK, ks > 0);
-        }
-        mma_commit(&bars->sdp_full);
-        ok = mbar_wait(&bars->ds_ready, s & 1, p.wait_ns, abort_flag, 213);
-        if (!ok) break;
-        tc_fence_after();
-        // dV += P^T dO ; dK += dS^T Q  (K dimension = the 128 queries of the step)
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          const uint32_t acc = (s > 0 || ks > 0) ? 1u : 0u;
-          mma_ts(tmem + C::COL_DV, tmem + C::COL_S + ks * 8, sdesc_sw128(sO + ks * 2048, 128 * 128, 1024), idTS,
+        for (int ks = 0; ks < 4; ++ks) {
+          const uint32_t acc = (s > 0 || hf > 0 || ks > 0) ? 1u : 0u;
+          const uint32_t roff = (hf * 4 + ks) * 2048;  // 16 query rows per k-step
+          mma_ts(tmem + C::COL_DV, tmem + C::COL_S + 64 * hf + ks * 8, sdesc_sw128(sO + roff, 128 * 128, 1024), idTS,
                  acc);
-          mma_ts(tmem + C::COL_DK, tmem + C::COL_DP + ks * 8, sdesc_sw128(sQ + ks * 2048, 128 * 128, 1024), idTS,
-                 acc);
+          mma_ts(tmem + C::COL_DK, tmem + C::COL_DP + 64 * hf + ks * 8, sdesc_sw128(sQ + roff, 128 * 128, 1024),
+                 idTS, acc);
         }
+      };
+      // dQ_i = dS K_j (M = queries, K dimension = the 128 keys); then release Q_i, dO_i
+      auto issue_dq = [&](int s) -> bool {
         const int qb = (C::NQB == 2) ? (s & 1) : 0;
         if constexpr (D == 64) {
-          if (s >= 2 && !(ok = mbar_wait(&bars->dq_free[qb], ((s >> 1) - 1) & 1, p.wait_ns, abort_flag, 214)))
-            break;
+          if (s >= 2 && !mbar_wait(&bars->dq_free[qb], ((s >> 1) - 1) & 1, p.wait_ns, abort_flag, 214)) return false;
         }
-        // dQ_i = dS K_j  (M = queries, K dimension = the 128 keys)
+        const uint32_t sds = sbase + C::OFF_DS + (s % C::DS_BUF) * (128 * 128 * 2);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
-          mma_ss(tmem + C::col_dq(qb), sdesc_sw128(sbase + C::OFF_DS + ks * 2048, 128 * 128, 1024),
+          mma_ss(tmem + C::col_dq(qb), sdesc_sw128(sds + ks * 2048, 128 * 128, 1024),
                  sdesc_sw128(sbase + C::OFF_K + ks * 2048, 128 * 128, 1024), idQ, ks > 0);
         mma_commit(&bars->dq_full[qb]);
-        mma_commit(&bars->qdo_empty[st]);
+        mma_commit(&bars->qdo_empty[s & 1]);
+        return true;
+      };
+      auto wait_qdo = [&](int s) { return mbar_wait(&bars->qdo_full[s & 1], (s >> 1) & 1, p.wait_ns, abort_flag, 211); };
+      auto wait_ds = [&](int s, int hf) { return mbar_wait(&bars->ds_ready[hf], s & 1, p.wait_ns, abort_flag, 213); };
+
+      bool ok = mbar_wait(&bars->kv_full, 0, p.wait_ns, abort_flag, 210);
+      if constexpr (C::EARLY) {
+        // half A of step s+1 enters the tensor core as soon as half A of step s is
+        // consumed, so the two softmax warpgroups run staggered by half a step
+        if (ok && (ok = wait_qdo(0))) {
+          tc_fence_after();
+          issue_sdp(0, 0);
+          issue_sdp(0, 1);
+        }
+        for (int s = 0; s < n_steps && ok; ++s) {
+          if (!(ok = wait_ds(s, 0))) break;
+          tc_fence_after();
+          issue_dvdk(s, 0);
+          if (s + 1 < n_steps) {
+            if (!(ok = wait_qdo(s + 1))) break;
+            tc_fence_after();
+            issue_sdp(s + 1, 0);
+          }
+          if (!(ok = wait_ds(s, 1))) break;
+          tc_fence_after();
+          issue_dvdk(s, 1);
+          if (!(ok = issue_dq(s))) break;
+          if (s + 1 < n_steps) issue_sdp(s + 1, 1);
+        }
+      } else {
+        for (int s = 0; s < n_steps && ok; ++s) {
+          if (!(ok = wait_qdo(s))) break;
+          if (s > 0 && !(ok = mbar_wait(&bars->dq_free[0], (s - 1) & 1, p.wait_ns, abort_flag, 212))) break;
+          tc_fence_after();  // (dP^T overwrites the previous dQ: its drain was awaited above)
+          issue_sdp(s, 0);
+          issue_sdp(s, 1);
+          for (int hf = 0; hf < 2 && ok; ++hf) {
+            if (!(ok = wait_ds(s, hf))) break;
+            tc_fence_after();
+            issue_dvdk(s, hf);
+          }
+          if (!ok || !(ok = issue_dq(s))) break;
+        }
       }
       if (ok) mma_commit(&bars->dkdv_full);
     }
-  } else if (warp >= 4 && warp < 8) {
-    // ---------------------------------------------------------------- softmax-gradient (key rows)
+  } else if (warp >= 4 && warp < 12) {
+    // ---------------------------------------------------------------- softmax-gradient
+    // warps 4-7: query half A (columns 0-63), warps 8-11: half B; one thread per key
+    const int hf = (warp - 4) >> 2;
     const int wq = warp & 3;
     const int r = wq * 32 + lane;  // key within the tile == TMEM lane
     const int key = k0 + r;
     const uint32_t lane_off = uint32_t(wq * 32) << 16;
+    const uint32_t cS = C::COL_S + 64 * hf, cDP = C::COL_DP + 64 * hf;
     const float sl2 = p.scale_log2, scale = p.scale;
     bool ok = true;
     for (int s = 0; s < n_steps && ok; ++s) {
       const int st = s & 1;
       const int i = i_begin + s % n_i;
-      ok = warp_wait(&bars->sdp_full, s & 1, p.wait_ns, abort_flag, 220) &&
+      ok = warp_wait(&bars->sdp_full[hf], s & 1, p.wait_ns, abort_flag, 220) &&
            warp_wait(&bars->qdo_full[st], (s >> 1) & 1, p.wait_ns, abort_flag, 221);
       if (!ok) break;
       tc_fence_after();
-      // columns q < lim are masked for this key (causal); a key past Nkv masks everything
+      // columns (queries of this half) q < lim are masked for this key; a key past Nkv
+      // masks everything
       int lim = 0;
-      if (key >= p.Nkv) lim = 128;
-      else if (CAUSAL) lim = min(128, max(0, key - off - i * C::BM));
-      const float* lse_s = reinterpret_cast<const float*>(smem + C::OFF_STAT + st * 1024);
+      if (key >= p.Nkv) lim = 64;
+      else if (CAUSAL) lim = min(64, max(0, key - off - i * C::BM - 64 * hf));
+      const float* lse_s = reinterpret_cast<const float*>(smem + C::OFF_STAT + st * 1024) + 64 * hf;
       const float* d_s = lse_s + 128;
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      const bool any_masked = __any_sync(0xffffffffu, lim > 0);
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
         uint32_t sv[32], dv[32];
-        tmem_ld32(tmem + lane_off + C::COL_S + c * 32, sv);
-        tmem_ld32(tmem + lane_off + C::COL_DP + c * 32, dv);
+        tmem_ld32(tmem + lane_off + cS + c * 32, sv);
+        tmem_ld32(tmem + lane_off + cDP + c * 32, dv);
         tmem_wait_ld();
         uint32_t pp[16], pd[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 4) {
           const float4 l4 = *reinterpret_cast<const float4*>(lse_s + c * 32 + e);
           const float4 d4 = *reinterpret_cast<const float4*>(d_s + c * 32 + e);
-          const float la[4] = {l4.x, l4.y, l4.z, l4.w}, da[4] = {d4.x, d4.y, d4.z, d4.w};
-          float pv[4], dsv[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            float pr = ex2(fmaf(__uint_as_float(sv[e + u]), sl2, -la[u]));
-            if (c * 32 + e + u < lim) pr = 0.f;
-            pv[u] = pr;
-            dsv[u] = pr * (__uint_as_float(dv[e + u]) - da[u]) * scale;
+          const float2 x01 = __ffma2_rn(make_float2(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])),
+                                        make_float2(sl2, sl2), make_float2(-l4.x, -l4.y));
+          const float2 x23 = __ffma2_rn(make_float2(__uint_as_float(sv[e + 2]), __uint_as_float(sv[e + 3])),
+                                        make_float2(sl2, sl2), make_float2(-l4.z, -l4.w));
+          float2 p01 = make_float2(ex2(x01.x), ex2(x01.y));
+          float2 p23 = make_float2(ex2(x23.x), ex2(x23.y));
+          if (any_masked) {
+            const int q0 = c * 32 + e;
+            if (q0 < lim) p01.x = 0.f;
+            if (q0 + 1 < lim) p01.y = 0.f;
+            if (q0 + 2 < lim) p23.x = 0.f;
+            if (q0 + 3 < lim) p23.y = 0.f;
           }
-          pp[e / 2] = pack_bf16x2(pv[0], pv[1]);
-          pp[e / 2 + 1] = pack_bf16x2(pv[2], pv[3]);
-          pd[e / 2] = pack_bf16x2(dsv[0], dsv[1]);
-          pd[e / 2 + 1] = pack_bf16x2(dsv[2], dsv[3]);
+          const float2 g01 = __fmul2_rn(p01, __fadd2_rn(make_float2(__uint_as_float(dv[e]), __uint_as_float(dv[e + 1])),
+                                                        make_float2(-d4.x, -d4.y)));
+          const float2 g23 = __fmul2_rn(p23, __fadd2_rn(make_float2(__uint_as_float(dv[e + 2]), __uint_as_float(dv[e + 3])),
+                                                        make_float2(-d4.z, -d4.w)));
+          pp[e / 2] = pack_bf16x2(p01.x, p01.y);
+          pp[e / 2 + 1] = pack_bf16x2(p23.x, p23.y);
+          pd[e / 2] = pack_bf16x2(g01.x * scale, g01.y * scale);
+          pd[e / 2 + 1] = pack_bf16x2(g23.x * scale, g23.y * scale);
         }
-        tmem_st16(tmem + lane_off + C::COL_S + c * 16, pp);
-        tmem_st16(tmem + lane_off + C::COL_DP + c * 16, pd);
-        // dS (query-major, 128-byte swizzle): queries [32c, 32c+32) = four 16-byte units
-        uint8_t* dsrow = smem + C::OFF_DS + (c >> 1) * (128 * 128) + r * 128;
+        tmem_st16(tmem + lane_off + cS + c * 16, pp);
+        tmem_st16(tmem + lane_off + cDP + c * 16, pd);
+        // dS (query-major, 128-byte swizzle): this half's queries form block hf
+        uint8_t* dsrow = smem + C::OFF_DS + (s % C::DS_BUF) * (128 * 128 * 2) + hf * (128 * 128) + r * 128;
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          const int unit = (c & 1) * 4 + u;
+          const int unit = c * 4 + u;
           *reinterpret_cast<uint4*>(dsrow + ((unit ^ (r & 7)) * 16)) =
               make_uint4(pd[4 * u], pd[4 * u + 1], pd[4 * u + 2], pd[4 * u + 3]);
         }
@@ -357,55 +421,48 @@ __global__ void __launch_bounds__(384, 1)
       fence_proxy_async_smem();  // dS written by the generic proxy, read by the tensor core
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->ds_ready);
+      if (lane == 0) mbar_arrive(&bars->ds_ready[hf]);
     }
-    // ---- dK_j, dV_j (scale already folded into dS)
+    // ---- dK_j (half A warps) and dV_j (half B warps); scale already folded into dS
+    const uint32_t col = hf == 0 ? C::COL_DK : C::COL_DV;
+    void* dst = hf == 0 ? p.dk : p.dv;
+    const size_t base = (size_t(bk) * p.Nkv + key) * D;
     if (ok && n_steps > 0) ok = warp_wait(&bars->dkdv_full, 0, p.wait_ns, abort_flag, 222);
     if (ok && n_steps > 0) {
       tc_fence_after();
 #pragma unroll 1
-      for (int which = 0; which < 2; ++which) {
-        const uint32_t col = which == 0 ? C::COL_DK : C::COL_DV;
-        void* dst = which == 0 ? p.dk : p.dv;
-        const size_t base = (size_t(bk) * p.Nkv + key) * D;
-#pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t v[32];
-          tmem_ld32(tmem + lane_off + col + c * 32, v);
-          tmem_wait_ld();
-          if (key < p.Nkv) {
-            if (p.grad_bf16) {
-              uint4* o4 = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(dst) + base + c * 32);
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tmem + lane_off + col + c * 32, v);
+        tmem_wait_ld();
+        if (key < p.Nkv) {
+          if (p.grad_bf16) {
+            uint4* o4 = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(dst) + base + c * 32);
 #pragma unroll
-              for (int q4 = 0; q4 < 4; ++q4)
-                o4[q4] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * q4]), __uint_as_float(v[8 * q4 + 1])),
-                                    pack_bf16x2(__uint_as_float(v[8 * q4 + 2]), __uint_as_float(v[8 * q4 + 3])),
-                                    pack_bf16x2(__uint_as_float(v[8 * q4 + 4]), __uint_as_float(v[8 * q4 + 5])),
-                                    pack_bf16x2(__uint_as_float(v[8 * q4 + 6]), __uint_as_float(v[8 * q4 + 7])));
-            } else {
-              float4* o4 = reinterpret_cast<float4*>(static_cast<float*>(dst) + base + c * 32);
+            for (int q4 = 0; q4 < 4; ++q4)
+              o4[q4] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * q4]), __uint_as_float(v[8 * q4 + 1])),
+                                  pack_bf16x2(__uint_as_float(v[8 * q4 + 2]), __uint_as_float(v[8 * q4 + 3])),
+                                  pack_bf16x2(__uint_as_float(v[8 * q4 + 4]), __uint_as_float(v[8 * q4 + 5])),
+                                  pack_bf16x2(__uint_as_float(v[8 * q4 + 6]), __uint_as_float(v[8 * q4 + 7])));
+          } else {
+            float4* o4 = reinterpret_cast<float4*>(static_cast<float*>(dst) + base + c * 32);
 #pragma unroll
-              for (int q4 = 0; q4 < 8; ++q4)
-                o4[q4] = make_float4(__uint_as_float(v[4 * q4]), __uint_as_float(v[4 * q4 + 1]),
-                                     __uint_as_float(v[4 * q4 + 2]), __uint_as_float(v[4 * q4 + 3]));
-            }
+            for (int q4 = 0; q4 < 8; ++q4)
+              o4[q4] = make_float4(__uint_as_float(v[4 * q4]), __uint_as_float(v[4 * q4 + 1]),
+                                   __uint_as_float(v[4 * q4 + 2]), __uint_as_float(v[4 * q4 + 3]));
           }
         }
       }
     } else if (n_steps == 0 && key < p.Nkv) {
       // no query row can see these keys: their gradients are zero
-      const size_t base = (size_t(bk) * p.Nkv + key) * D;
       for (int c = 0; c < D; c += 4) {
-        if (p.grad_bf16) {
-          *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.dk) + base + c) = make_uint2(0, 0);
-          *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.dv) + base + c) = make_uint2(0, 0);
-        } else {
-          *reinterpret_cast<float4*>(static_cast<float*>(p.dk) + base + c) = make_float4(0, 0, 0, 0);
-          *reinterpret_cast<float4*>(static_cast<float*>(p.dv) + base + c) = make_float4(0, 0, 0, 0);
-        }
+        if (p.grad_bf16)
+          *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(dst) + base + c) = make_uint2(0, 0);
+        else
+          *reinterpret_cast<float4*>(static_cast<float*>(dst) + base + c) = make_float4(0, 0, 0, 0);
       }
     }
-  } else if (warp >= 8) {
+  } else if (warp >= 12) {
     // ---------------------------------------------------------------- dQ drain (query rows)
     const int wq = warp & 3;
     const int r = wq * 32 + lane;
@@ -419,7 +476,7 @@ __global__ void __launch_bounds__(384, 1)
       tc_fence_after();
       const int h = hk * G + s / n_i, i = i_begin + s % n_i;
       const int q = i * C::BM + r;
-      float* dst = p.dq_acc + ((size_t(b) * p.Hq + h) * p.Nq + q) * D;
+      float* dstq = p.dq_acc + ((size_t(b) * p.Hq + h) * p.Nq + q) * D;
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         uint32_t v[32];
@@ -428,7 +485,7 @@ __global__ void __launch_bounds__(384, 1)
         if (q < p.Nq) {
 #pragma unroll
           for (int e = 0; e < 32; e += 4)
-            red_add_v4(dst + c * 32 + e, __uint_as_float(v[e]), __uint_as_float(v[e + 1]),
+            red_add_v4(dstq + c * 32 + e, __uint_as_float(v[e]), __uint_as_float(v[e + 1]),
                        __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
         }
       }
