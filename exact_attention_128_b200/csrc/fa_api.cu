@@ -11,6 +11,10 @@
 #include "fwd_f32.cuh"
 #include "bwd_bf16.cuh"
 
+#ifndef FA_FWD_D64_BN
+#define FA_FWD_D64_BN 64
+#endif
+
 namespace {
 
 using namespace fa;
@@ -80,16 +84,16 @@ int sm_count() {
   return n;
 }
 
-template <int D, bool CAUSAL>
+template <int D, int BN, bool CAUSAL>
 fa_status launch_fwd_bf16(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                          const FwdBf16Params& prm, int Nq, cudaStream_t st) {
-  using C = FwdCfg<D>;
-  auto kern = fa_fwd_bf16_kernel<D, CAUSAL>;
+                          const CUtensorMap& mo, const FwdBf16Params& prm, int Nq, cudaStream_t st) {
+  using C = FwdCfg<D, BN>;
+  auto kern = fa_fwd_bf16_kernel<D, BN, CAUSAL>;
   if (set_smem(kern, C::SMEM) != cudaSuccess) return FA_ERR_CUDA;
   const long items = long((Nq + 2 * C::BM - 1) / (2 * C::BM)) * prm.BH;
-  const int sms = sm_count();
-  if (sms <= 0) return FA_ERR_CUDA;
-  kern<<<int(items < sms ? items : sms), C::THREADS, C::SMEM, st>>>(mq, mk, mv, prm);
+  const long slots = long(sm_count()) * C::CTAS_PER_SM;
+  if (slots <= 0) return FA_ERR_CUDA;
+  kern<<<int(items < slots ? items : slots), C::THREADS, C::SMEM, st>>>(mq, mk, mv, mo, prm);
   return launched();
 }
 
@@ -246,17 +250,19 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   if (dtype != FA_DTYPE_BF16) return FA_ERR_UNSUPPORTED;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
 
-  CUtensorMap mq, mk, mv;
-  if (!make_map_bf16(&mq, q, d, Nq, B * Hq, 128) || !make_map_bf16(&mk, k, d, Nkv, B * Hkv, 128) ||
-      !make_map_bf16(&mv, v, d, Nkv, B * Hkv, 128))
+  constexpr int BN64 = FA_FWD_D64_BN;  // key-tile width of the d = 64 kernel
+  const int bn = d == 64 ? BN64 : 128;
+  CUtensorMap mq, mk, mv, mo;
+  if (!make_map_bf16(&mq, q, d, Nq, B * Hq, 128) || !make_map_bf16(&mk, k, d, Nkv, B * Hkv, bn) ||
+      !make_map_bf16(&mv, v, d, Nkv, B * Hkv, bn) || !make_map_bf16(&mo, o, d, Nq, B * Hq, 32))
     return FA_ERR_CUDA;
   FwdBf16Params prm{static_cast<__nv_bfloat16*>(o), lse, B * Hq, Hq, Hkv, Nq, Nkv,
                     scale * 1.4426950408889634f, g_wait_ns};
   if (d == 64)
-    return causal ? launch_fwd_bf16<64, true>(mq, mk, mv, prm, Nq, st)
-                  : launch_fwd_bf16<64, false>(mq, mk, mv, prm, Nq, st);
-  return causal ? launch_fwd_bf16<128, true>(mq, mk, mv, prm, Nq, st)
-                : launch_fwd_bf16<128, false>(mq, mk, mv, prm, Nq, st);
+    return causal ? launch_fwd_bf16<64, BN64, true>(mq, mk, mv, mo, prm, Nq, st)
+                  : launch_fwd_bf16<64, BN64, false>(mq, mk, mv, mo, prm, Nq, st);
+  return causal ? launch_fwd_bf16<128, 128, true>(mq, mk, mv, mo, prm, Nq, st)
+                : launch_fwd_bf16<128, 128, false>(mq, mk, mv, mo, prm, Nq, st);
 }
 
 size_t fa_bwd_workspace_size(int B, int Hq, int Nq, int d) {

@@ -41,24 +41,33 @@ namespace fa {
 #define FWD_EMU_PAIRS 0x00u
 #endif
 
-template <int D>
+// Two configurations:
+//   BN = 128 (d = 128): 384 threads (softmax warps 4-11), 512 TMEM columns, one CTA/SM.
+//   BN = 64  (d = 64):  320 threads (softmax warps 2-9), 256 TMEM columns and ~97 KB of
+//            shared memory, so two CTAs share an SM and four query tiles are in flight;
+//            at d = 64 the softmax, not the tensor core, sets the pace, and the second
+//            CTA hides its latency.
+template <int D, int BN_>
 struct FwdCfg {
-  static constexpr int BM = 128;  // rows per query tile (two tiles per item)
-  static constexpr int BN = 128;  // keys per tile
+  static constexpr int BM = 128;   // rows per query tile (two tiles per item)
+  static constexpr int BN = BN_;   // keys per tile
   static constexpr int KB = D / 64;
   static constexpr int Q_TILE = BM * D * 2;
   static constexpr int KV_TILE = BN * D * 2;
-  static constexpr int QBUF = (D == 128) ? 1 : 2;
-  static constexpr int NSTAGE = (D == 128) ? 2 : 4;
+  static constexpr int QBUF = (D == 128 || BN == 64) ? 1 : 2;
+  static constexpr int NSTAGE = (BN == 64) ? 2 : (D == 128 ? 2 : 4);
   static constexpr int OFF_Q = 0;  // + qb * 2 * Q_TILE + t * Q_TILE
   static constexpr int OFF_K = QBUF * 2 * Q_TILE;
   static constexpr int OFF_V = OFF_K + NSTAGE * KV_TILE;
-  static constexpr int OFF_BAR = OFF_V + NSTAGE * KV_TILE;
+  static constexpr int OFF_STG = OFF_V + NSTAGE * KV_TILE;  // epilogue staging: 4 KB per softmax warp
+  static constexpr int OFF_BAR = OFF_STG + 8 * 4096;
   static constexpr int SMEM = OFF_BAR + 256 + 1024;  // + barriers + alignment slack
-  static constexpr int THREADS = 384;
-  static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t COL_S = 0;    // + t * 128
-  static constexpr uint32_t COL_O = 256;  // + t * D
+  static constexpr int WG0 = (BN == 64) ? 2 : 4;     // first softmax warp
+  static constexpr int THREADS = 32 * (WG0 + 8);
+  static constexpr int CTAS_PER_SM = (BN == 64) ? 2 : 1;
+  static constexpr uint32_t TMEM_COLS = (BN == 64) ? 256 : 512;
+  static constexpr uint32_t COL_S = 0;       // + t * BN
+  static constexpr uint32_t COL_O = 2 * BN;  // + t * D
 };
 
 struct FwdBf16Params {
@@ -82,11 +91,12 @@ struct FwdBars {
   int abort_flag;
 };
 
-template <int D, bool CAUSAL>
-__global__ void __launch_bounds__(384, 1)
+template <int D, int BN, bool CAUSAL>
+__global__ void __launch_bounds__(FwdCfg<D, BN>::THREADS, FwdCfg<D, BN>::CTAS_PER_SM)
     fa_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                       const __grid_constant__ CUtensorMap tmV, const FwdBf16Params p) {
-  using C = FwdCfg<D>;
+                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                       const FwdBf16Params p) {
+  using C = FwdCfg<D, BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   FwdBars* bars = reinterpret_cast<FwdBars*>(smem + C::OFF_BAR);
@@ -184,14 +194,14 @@ __global__ void __launch_bounds__(384, 1)
           const uint64_t a =
               sdesc_sw128(sQ + (qb * 2 + t) * C::Q_TILE + kb * C::BM * 128 + kin * 32, 16, 1024);
           const uint64_t bd = sdesc_sw128(sK + st * C::KV_TILE + kb * C::BN * 128 + kin * 32, 16, 1024);
-          mma_ss(tmem + C::COL_S + t * 128, a, bd, idS, ks > 0 ? 1u : 0u);
+          mma_ss(tmem + C::COL_S + t * C::BN, a, bd, idS, ks > 0 ? 1u : 0u);
         }
       };
       auto issue_PV = [&](int t, int st, int j) {
 #pragma unroll
         for (int ks = 0; ks < C::BN / 16; ++ks) {
           const uint64_t bd = sdesc_sw128(sV + st * C::KV_TILE + ks * 16 * 128, C::BN * 128, 1024);
-          mma_ts(tmem + C::COL_O + t * D, tmem + C::COL_S + t * 128 + ks * 8, bd, idPV,
+          mma_ts(tmem + C::COL_O + t * D, tmem + C::COL_S + t * C::BN + ks * 8, bd, idPV,
                  (j > 0 || ks > 0) ? 1u : 0u);
         }
       };
@@ -243,13 +253,13 @@ __global__ void __launch_bounds__(384, 1)
         }
       }
     }
-  } else if (warp >= 4) {
+  } else if (warp >= C::WG0) {
     // ---------------------------------------------------------------- softmax + epilogue
-    const int t = (warp - 4) >> 2;              // which query tile
+    const int t = (warp - C::WG0) >> 2;         // which query tile
     const int wq = warp & 3;                    // TMEM lane quarter this warp may access
     const int r = wq * 32 + lane;               // row within the tile == TMEM lane
     const uint32_t lane_off = uint32_t(wq * 32) << 16;
-    const uint32_t tS = tmem + lane_off + C::COL_S + t * 128;
+    const uint32_t tS = tmem + lane_off + C::COL_S + t * C::BN;
     const uint32_t tO = tmem + lane_off + C::COL_O + t * D;
     const float sl2 = p.scale_log2;
     int g = 0, local = 0;
@@ -363,26 +373,43 @@ __global__ void __launch_bounds__(384, 1)
       if (!ok) break;
       if (idle) continue;
       tc_fence_after();
+      // O = u / l, staged per warp (32 rows x 64 columns, 128-byte swizzle) and written by
+      // a TMA store, which also drops the rows past Nq
       const float inv = 1.f / l;
-      __nv_bfloat16* orow = p.o + (size_t(bh) * p.Nq + row) * D;
+      uint8_t* stg = smem + C::OFF_STG + (warp - C::WG0) * 4096;
+      const int row0 = qt * 2 * C::BM + t * C::BM + wq * 32;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t o[32];
-        tmem_ld32(tO + c * 32, o);
+      for (int c = 0; c < D / 64; ++c) {
+        uint32_t o[64];
+        tmem_ld32(tO + c * 64, *reinterpret_cast<uint32_t(*)[32]>(&o[0]));
+        tmem_ld32(tO + c * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&o[32]));
         tmem_wait_ld();
-        uint32_t pk[16];
+        if (lane == 0) bulk_wait_read();  // the previous store from this staging buffer
+        __syncwarp();
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          pk[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
-        if (row < p.Nq) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
-#pragma unroll
-          for (int v4 = 0; v4 < 4; ++v4)
-            dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+        for (int u = 0; u < 8; ++u) {
+          const float2 a = __fmul2_rn(make_float2(__uint_as_float(o[8 * u]), __uint_as_float(o[8 * u + 1])),
+                                      make_float2(inv, inv));
+          const float2 b2 = __fmul2_rn(make_float2(__uint_as_float(o[8 * u + 2]), __uint_as_float(o[8 * u + 3])),
+                                       make_float2(inv, inv));
+          const float2 c2 = __fmul2_rn(make_float2(__uint_as_float(o[8 * u + 4]), __uint_as_float(o[8 * u + 5])),
+                                       make_float2(inv, inv));
+          const float2 d2 = __fmul2_rn(make_float2(__uint_as_float(o[8 * u + 6]), __uint_as_float(o[8 * u + 7])),
+                                       make_float2(inv, inv));
+          *reinterpret_cast<uint4*>(stg + lane * 128 + ((u ^ (lane & 7)) << 4)) =
+              make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(b2.x, b2.y), pack_bf16x2(c2.x, c2.y),
+                         pack_bf16x2(d2.x, d2.y));
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_3d(&tmO, stg, c * 64, row0, bh);
+          bulk_commit();
         }
       }
       if (row < p.Nq) p.lse[size_t(bh) * p.Nq + row] = (m + __log2f(l)) * 0.69314718055994531f;
     }
+    if (lane == 0) bulk_wait_all();
   }
 
   tc_fence_before();
