@@ -55,7 +55,12 @@ struct BwdCfg {
   static constexpr int DS_BUF = EARLY ? 2 : 1;
   static constexpr int OFF_DS = OFF_DO + 2 * TILE;     // DS_BUF x [2 query chunks][128 keys][128 B]
   static constexpr int OFF_STAT = OFF_DS + DS_BUF * 128 * 128 * 2;  // per stage: lse2[128], D[128]
-  static constexpr int OFF_BAR = OFF_STAT + 2 * 2 * 512;
+  // d = 64 adds dQ into the fp32 accumulator with TMA reduce-adds from per-warp staging
+  // (4 drain warps x 32 rows x 64 fp32, 128-byte swizzle); d = 128 has no room left and
+  // uses vector reductions from registers
+  static constexpr bool DQ_TMA = (D == 64);
+  static constexpr int OFF_DQS = OFF_STAT + 2 * 2 * 512;
+  static constexpr int OFF_BAR = OFF_DQS + (DQ_TMA ? 4 * 32 * 64 * 4 : 0);
   // D = 128 fills the 227 KB limit exactly, leaving no room to re-align the base: that
   // variant relies on the dynamic shared memory starting 1024-byte aligned and checks it.
   static constexpr int SLACK = (D == 128) ? 0 : 1024;
@@ -167,8 +172,8 @@ template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(512, 1)
     fa_bwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
-                       const BwdParams p) {
-  // tmO maps dO (same geometry as Q)
+                       const __grid_constant__ CUtensorMap tmDQ, const BwdParams p) {
+  // tmO maps dO (same geometry as Q); tmDQ maps the fp32 dQ accumulator (32 x 32 boxes)
   using C = BwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   if (C::SLACK == 0 && (smem_u32(smem_raw) & 1023u) != 0) {  // uniform across the CTA
@@ -476,23 +481,48 @@ __global__ void __launch_bounds__(512, 1)
       tc_fence_after();
       const int h = hk * G + s / n_i, i = i_begin + s % n_i;
       const int q = i * C::BM + r;
-      float* dstq = p.dq_acc + ((size_t(b) * p.Hq + h) * p.Nq + q) * D;
-#pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tmem + lane_off + C::col_dq(qb) + c * 32, v);
+      if constexpr (C::DQ_TMA) {
+        uint8_t* stg = smem + C::OFF_DQS + wq * (32 * 64 * 4);  // two 32x32 fp32 boxes
+        uint32_t v[64];
+        tmem_ld32(tmem + lane_off + C::col_dq(qb), *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+        tmem_ld32(tmem + lane_off + C::col_dq(qb) + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
         tmem_wait_ld();
-        if (q < p.Nq) {
+        if (lane == 0) bulk_wait_read();  // this warp's previous reduce has read the staging
+        __syncwarp();
 #pragma unroll
-          for (int e = 0; e < 32; e += 4)
-            red_add_v4(dstq + c * 32 + e, __uint_as_float(v[e]), __uint_as_float(v[e + 1]),
-                       __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+        for (int hb = 0; hb < 2; ++hb)
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            *reinterpret_cast<uint4*>(stg + hb * 4096 + lane * 128 + ((u ^ (lane & 7)) << 4)) =
+                make_uint4(v[32 * hb + 4 * u], v[32 * hb + 4 * u + 1], v[32 * hb + 4 * u + 2], v[32 * hb + 4 * u + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          const int row0 = i * C::BM + wq * 32, z = b * p.Hq + h;
+          tma_reduce_add_3d(&tmDQ, stg, 0, row0, z);
+          tma_reduce_add_3d(&tmDQ, stg + 4096, 32, row0, z);
+          bulk_commit();
+        }
+      } else {
+        float* dstq = p.dq_acc + ((size_t(b) * p.Hq + h) * p.Nq + q) * D;
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tmem + lane_off + C::col_dq(qb) + c * 32, v);
+          tmem_wait_ld();
+          if (q < p.Nq) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 4)
+              red_add_v4(dstq + c * 32 + e, __uint_as_float(v[e]), __uint_as_float(v[e + 1]),
+                         __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+          }
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->dq_free[qb]);
     }
+    if (C::DQ_TMA && lane == 0) bulk_wait_all();  // the reduce-adds complete before exit
   }
 
   tc_fence_before();

@@ -10,7 +10,8 @@
 // ("Mecanismo y detalles", GQA) are processed together, so each K/V byte is read once.
 //
 // Work split (split-KV): CTA (split s, kv head g, request r) covers logical blocks
-// [s*CHUNK, (s+1)*CHUNK) of request r.  Each of its 4 warps takes every 4th block and
+// [s*CHUNK, (s+1)*CHUNK) of request r (CHUNK = 64 blocks = 1024 tokens by default).  Each
+// of its 4 warps takes every 4th block and
 // keeps its own (m, l, u) state; the warps' states and then the splits' partial
 // results are merged by weighting each part with its unnormalised mass e^{lse_s}
 // ("No basta con promediar los resultados de los bloques": block results are never
@@ -29,9 +30,16 @@ namespace fa {
 namespace dec {
 constexpr int D = 128;
 constexpr int BS = 16;          // tokens per cache block
+#ifndef FA_DEC_STAGES
+#define FA_DEC_STAGES 3
+#endif
+#ifndef FA_DEC_CHUNK
+#define FA_DEC_CHUNK 64
+#endif
 constexpr int WARPS = 4;
-constexpr int STAGES = 3;       // blocks in flight per warp
-constexpr int CHUNK = 32;       // logical blocks per CTA (split size = 512 tokens)
+constexpr int STAGES = FA_DEC_STAGES;  // blocks in flight per warp
+constexpr int CHUNK = FA_DEC_CHUNK;    // logical blocks per CTA (split size = CHUNK * 16 tokens)
+static_assert(CHUNK / WARPS <= 32, "a warp's block-table entries are held one per lane");
 constexpr int SLAB = BS * D * 2;  // 4096 bytes: one (block, kv head) slab of K or V
 constexpr int STAGE_BYTES = 2 * SLAB;
 constexpr int OFF_BAR = WARPS * STAGES * STAGE_BYTES;

@@ -101,14 +101,28 @@ int round_up(int x, int m) { return (x + m - 1) / m * m; }
 
 template <int D, bool CAUSAL>
 fa_status launch_bwd_kernel(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                            const CUtensorMap& mo, const BwdParams& prm, int B, int Hkv, int Nkv,
-                            cudaStream_t st) {
+                            const CUtensorMap& mo, const CUtensorMap& mdq, const BwdParams& prm, int B, int Hkv,
+                            int Nkv, cudaStream_t st) {
   using C = BwdCfg<D>;
   auto kern = fa_bwd_bf16_kernel<D, CAUSAL>;
   if (set_smem(kern, C::SMEM) != cudaSuccess) return FA_ERR_CUDA;
   dim3 grid((Nkv + C::BN - 1) / C::BN, B * Hkv);
-  kern<<<grid, C::THREADS, C::SMEM, st>>>(mq, mk, mv, mo, prm);
+  kern<<<grid, C::THREADS, C::SMEM, st>>>(mq, mk, mv, mo, mdq, prm);
   return launched();
+}
+
+// 3-D fp32 map over the dQ accumulator [planes][rows][d] with a (32, 32, 1) box and the
+// 128-byte swizzle (for TMA reduce-adds).
+bool make_map_f32(CUtensorMap* m, const void* base, int d, int rows, int planes) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(rows), cuuint64_t(planes)};
+  cuuint64_t strides[2] = {cuuint64_t(d) * 4, cuuint64_t(d) * 4 * cuuint64_t(rows)};
+  cuuint32_t box[3] = {32, 32, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // Backward: preprocess (D, padded lse, zeroed dQ accumulator), the tensor-core kernel,
@@ -137,19 +151,20 @@ fa_status bwd_launch(const void* q, const void* k, const void* v, const void* o,
         long(rows_pad), Nq, Nq_pad, long(rows) * d);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
 
-  CUtensorMap mq, mk, mv, mo;
+  CUtensorMap mq, mk, mv, mo, mdq;
   if (!make_map_bf16(&mq, q, d, Nq, B * Hq, 128) || !make_map_bf16(&mk, k, d, Nkv, B * Hkv, 128) ||
-      !make_map_bf16(&mv, v, d, Nkv, B * Hkv, 128) || !make_map_bf16(&mo, dO, d, Nq, B * Hq, 128))
+      !make_map_bf16(&mv, v, d, Nkv, B * Hkv, 128) || !make_map_bf16(&mo, dO, d, Nq, B * Hq, 128) ||
+      !make_map_f32(&mdq, dq_acc, d, Nq, B * Hq))
     return FA_ERR_CUDA;
   BwdParams prm{dq_acc, lse2, dstat, dk, dv, grad_dtype == FA_DTYPE_BF16 ? 1 : 0, Hq, Hkv, Nq, Nkv, Nq_pad,
                 scale, scale * 1.4426950408889634f, g_wait_ns};
   fa_status s;
   if (d == 64)
-    s = causal ? launch_bwd_kernel<64, true>(mq, mk, mv, mo, prm, B, Hkv, Nkv, st)
-               : launch_bwd_kernel<64, false>(mq, mk, mv, mo, prm, B, Hkv, Nkv, st);
+    s = causal ? launch_bwd_kernel<64, true>(mq, mk, mv, mo, mdq, prm, B, Hkv, Nkv, st)
+               : launch_bwd_kernel<64, false>(mq, mk, mv, mo, mdq, prm, B, Hkv, Nkv, st);
   else
-    s = causal ? launch_bwd_kernel<128, true>(mq, mk, mv, mo, prm, B, Hkv, Nkv, st)
-               : launch_bwd_kernel<128, false>(mq, mk, mv, mo, prm, B, Hkv, Nkv, st);
+    s = causal ? launch_bwd_kernel<128, true>(mq, mk, mv, mo, mdq, prm, B, Hkv, Nkv, st)
+               : launch_bwd_kernel<128, false>(mq, mk, mv, mo, mdq, prm, B, Hkv, Nkv, st);
   if (s != FA_OK) return s;
   if (grad_dtype == FA_DTYPE_BF16) {
     const long n = long(rows) * d;
