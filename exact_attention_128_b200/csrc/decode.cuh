@@ -113,7 +113,10 @@ __global__ void __launch_bounds__(dec::WARPS * 32)
   const int nblk = (ctx + BS - 1) / BS;
   const int nsplit = (nblk + CHUNK - 1) / CHUNK;
   const int b0 = s * CHUNK;
-  if (b0 >= nblk) return;
+  if (b0 >= nblk) {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    return;
+  }
   const int b1 = min(nblk, b0 + CHUNK);
 
   const int warp = warp_id(), lane = lane_id();
@@ -309,12 +312,17 @@ __global__ void __launch_bounds__(dec::WARPS * 32)
       if (d == 0) p.part_lse[pi] = lse_nat;
     }
   }
+  // the merge kernel (launched as a programmatic dependent) may start scheduling now; it
+  // waits for this grid's completion and memory before reading the partials
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // Merge the split partials of requests that needed more than one split: each split's
 // normalised output is weighted by e^{lse_s - lse}, lse = ln sum_s e^{lse_s}.
 __global__ void __launch_bounds__(128) fa_paged_decode_combine_kernel(const DecodeParams p) {
   using namespace dec;
+  // launched with programmatic stream serialization: wait for the split kernel
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int rh = blockIdx.x;
   const int r = rh / p.Hq;
   const int ctx = p.ctx[r];

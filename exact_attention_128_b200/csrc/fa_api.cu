@@ -346,7 +346,19 @@ fa_status fa_paged_decode(const void* q, const void* k_cache, const void* v_cach
   if (set_smem(fa_paged_decode_kernel, dec::SMEM) != cudaSuccess) return FA_ERR_CUDA;
   fa_paged_decode_kernel<<<dim3(max_splits, Hkv, R), dec::WARPS * 32, dec::SMEM, st>>>(mk, mv, prm);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
-  fa_paged_decode_combine_kernel<<<R * Hq, dec::D, 0, st>>>(prm);
+  // the merge is a programmatic dependent launch: its launch overlaps the split kernel's
+  // tail and it waits (griddepcontrol.wait) for the split kernel's results
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(R * Hq);
+  cfg.blockDim = dim3(dec::D);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, fa_paged_decode_combine_kernel, prm) != cudaSuccess) return FA_ERR_CUDA;
   return launched();
 }
 
