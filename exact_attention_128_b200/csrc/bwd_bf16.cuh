@@ -21,10 +21,11 @@
 //        warp 1      MMA issuer (one thread): per half, S^T = K_j Q_h^T and dP^T = V_j dO_h^T
 //                    into TMEM; per half, dV += P^T dO_h and dK += dS^T Q_h with P^T, dS^T
 //                    read from TMEM; then dQ_i = dS K_j with dS read from shared memory.
-//        warps 4-7   half A, warps 8-11 half B; one thread per key (TMEM lane): P^T and
-//                    dS^T from S^T, dP^T, lse, D; P^T and dS^T (bf16) go back over S^T and
-//                    dP^T in TMEM, dS^T also to shared memory (swizzled, query-major) for
-//                    the dQ MMA.  At the end half A's warps write dK_j, half B's dV_j.
+//        warps 4-11  one thread per key (TMEM lane), both warpgroups on half A and then
+//                    on half B (32 columns each): P^T and dS^T from S^T, dP^T, lse, D;
+//                    P^T and dS^T (bf16) go back over S^T and dP^T in TMEM, dS^T also to
+//                    shared memory (swizzled, query-major) for the dQ MMA.  At the end
+//                    warps 4-7 write dK_j and warps 8-11 dV_j.
 //        warps 12-15 one thread per query row: read dQ_i from TMEM and add it into the fp32
 //                    accumulator with vector reductions (red.global.add.v4.f32).
 //   3. fa_bwd_finalize_kernel: fp32 dQ accumulator -> bf16 dq (only for bf16 gradients;
@@ -205,7 +206,7 @@ __global__ void __launch_bounds__(512, 1)
       mbar_init(&bars->dq_full[s], 1);
       mbar_init(&bars->dq_free[s], 4);
       mbar_init(&bars->sdp_full[s], 1);
-      mbar_init(&bars->ds_ready[s], 4);
+      mbar_init(&bars->ds_ready[s], 8);
     }
     mbar_init(&bars->dkdv_full, 1);
     bars->abort_flag = 0;
@@ -287,10 +288,9 @@ __global__ void __launch_bounds__(512, 1)
         for (int ks = 0; ks < 4; ++ks) {
           const uint32_t acc = (s > 0 || hf > 0 || ks > 0) ? 1u : 0u;
           const uint32_t roff = (hf * 4 + ks) * 2048;  // 16 query rows per k-step
-          mma_ts(tmem + C::COL_DV, tmem + C::COL_S + 64 * hf + ks * 8, sdesc_sw128(sO + roff, 128 * 128, 1024), idTS,
-                 acc);
-          mma_ts(tmem + C::COL_DK, tmem + C::COL_DP + 64 * hf + ks * 8, sdesc_sw128(sQ + roff, 128 * 128, 1024),
-                 idTS, acc);
+          const uint32_t pcol = 64 * hf + (ks >> 1) * 32 + (ks & 1) * 8;  // packed P / dS of queries 16ks..
+          mma_ts(tmem + C::COL_DV, tmem + C::COL_S + pcol, sdesc_sw128(sO + roff, 128 * 128, 1024), idTS, acc);
+          mma_ts(tmem + C::COL_DK, tmem + C::COL_DP + pcol, sdesc_sw128(sQ + roff, 128 * 128, 1024), idTS, acc);
         }
       };
       // dQ_i = dS K_j (M = queries, K dimension = the 128 keys); then release Q_i, dO_i
@@ -354,41 +354,42 @@ __global__ void __launch_bounds__(512, 1)
     }
   } else if (warp >= 4 && warp < 12) {
     // ---------------------------------------------------------------- softmax-gradient
-    // warps 4-7: query half A (columns 0-63), warps 8-11: half B; one thread per key
-    const int hf = (warp - 4) >> 2;
+    // Both warpgroups work on query half A, then both on half B: warps 4-7 take columns
+    // [0, 32) of the half and warps 8-11 columns [32, 64), so every half has two warps per
+    // SMSP to hide each other's latency.  One thread per key (TMEM lane).
+    const int wg = (warp - 4) >> 2;
     const int wq = warp & 3;
     const int r = wq * 32 + lane;  // key within the tile == TMEM lane
     const int key = k0 + r;
     const uint32_t lane_off = uint32_t(wq * 32) << 16;
-    const uint32_t cS = C::COL_S + 64 * hf, cDP = C::COL_DP + 64 * hf;
     const float sl2 = p.scale_log2, scale = p.scale;
     bool ok = true;
     for (int s = 0; s < n_steps && ok; ++s) {
       const int st = s & 1;
       const int i = i_begin + s % n_i;
-      ok = warp_wait(&bars->sdp_full[hf], s & 1, p.wait_ns, abort_flag, 220) &&
-           warp_wait(&bars->qdo_full[st], (s >> 1) & 1, p.wait_ns, abort_flag, 221);
-      if (!ok) break;
-      tc_fence_after();
-      // columns (queries of this half) q < lim are masked for this key; a key past Nkv
-      // masks everything
-      int lim = 0;
-      if (key >= p.Nkv) lim = 64;
-      else if (CAUSAL) lim = min(64, max(0, key - off - i * C::BM - 64 * hf));
-      const float* lse_s = reinterpret_cast<const float*>(smem + C::OFF_STAT + st * 1024) + 64 * hf;
-      const float* d_s = lse_s + 128;
-      const bool any_masked = __any_sync(0xffffffffu, lim > 0);
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
+      ok = warp_wait(&bars->qdo_full[st], (s >> 1) & 1, p.wait_ns, abort_flag, 221);
+#pragma unroll 1
+      for (int hf = 0; hf < 2 && ok; ++hf) {
+        ok = warp_wait(&bars->sdp_full[hf], s & 1, p.wait_ns, abort_flag, 220);
+        if (!ok) break;
+        tc_fence_after();
+        const int q0 = 64 * hf + 32 * wg;  // first query (column) of this thread's chunk
+        // columns q < lim of the chunk are masked for this key; a key past Nkv masks all
+        int lim = 0;
+        if (key >= p.Nkv) lim = 32;
+        else if (CAUSAL) lim = min(32, max(0, key - off - i * C::BM - q0));
+        const float* lse_s = reinterpret_cast<const float*>(smem + C::OFF_STAT + st * 1024) + q0;
+        const float* d_s = lse_s + 128;
+        const bool any_masked = __any_sync(0xffffffffu, lim > 0);
         uint32_t sv[32], dv[32];
-        tmem_ld32(tmem + lane_off + cS + c * 32, sv);
-        tmem_ld32(tmem + lane_off + cDP + c * 32, dv);
+        tmem_ld32(tmem + lane_off + C::COL_S + q0, sv);
+        tmem_ld32(tmem + lane_off + C::COL_DP + q0, dv);
         tmem_wait_ld();
         uint32_t pp[16], pd[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 4) {
-          const float4 l4 = *reinterpret_cast<const float4*>(lse_s + c * 32 + e);
-          const float4 d4 = *reinterpret_cast<const float4*>(d_s + c * 32 + e);
+          const float4 l4 = *reinterpret_cast<const float4*>(lse_s + e);
+          const float4 d4 = *reinterpret_cast<const float4*>(d_s + e);
           const float2 x01 = __ffma2_rn(make_float2(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])),
                                         make_float2(sl2, sl2), make_float2(-l4.x, -l4.y));
           const float2 x23 = __ffma2_rn(make_float2(__uint_as_float(sv[e + 2]), __uint_as_float(sv[e + 3])),
@@ -396,38 +397,46 @@ __global__ void __launch_bounds__(512, 1)
           float2 p01 = make_float2(ex2(x01.x), ex2(x01.y));
           float2 p23 = make_float2(ex2(x23.x), ex2(x23.y));
           if (any_masked) {
-            const int q0 = c * 32 + e;
-            if (q0 < lim) p01.x = 0.f;
-            if (q0 + 1 < lim) p01.y = 0.f;
-            if (q0 + 2 < lim) p23.x = 0.f;
-            if (q0 + 3 < lim) p23.y = 0.f;
+            if (e < lim) p01.x = 0.f;
+            if (e + 1 < lim) p01.y = 0.f;
+            if (e + 2 < lim) p23.x = 0.f;
+            if (e + 3 < lim) p23.y = 0.f;
           }
-          const float2 g01 = __fmul2_rn(p01, __fadd2_rn(make_float2(__uint_as_float(dv[e]), __uint_as_float(dv[e + 1])),
-                                                        make_float2(-d4.x, -d4.y)));
-          const float2 g23 = __fmul2_rn(p23, __fadd2_rn(make_float2(__uint_as_float(dv[e + 2]), __uint_as_float(dv[e + 3])),
-                                                        make_float2(-d4.z, -d4.w)));
+          // dS * scale = P * (dP - D) * scale
+          const float2 g01 = __fmul2_rn(
+              __fmul2_rn(p01, __fadd2_rn(make_float2(__uint_as_float(dv[e]), __uint_as_float(dv[e + 1])),
+                                         make_float2(-d4.x, -d4.y))),
+              make_float2(scale, scale));
+          const float2 g23 = __fmul2_rn(
+              __fmul2_rn(p23, __fadd2_rn(make_float2(__uint_as_float(dv[e + 2]), __uint_as_float(dv[e + 3])),
+                                         make_float2(-d4.z, -d4.w))),
+              make_float2(scale, scale));
           pp[e / 2] = pack_bf16x2(p01.x, p01.y);
           pp[e / 2 + 1] = pack_bf16x2(p23.x, p23.y);
-          pd[e / 2] = pack_bf16x2(g01.x * scale, g01.y * scale);
-          pd[e / 2 + 1] = pack_bf16x2(g23.x * scale, g23.y * scale);
+          pd[e / 2] = pack_bf16x2(g01.x, g01.y);
+          pd[e / 2 + 1] = pack_bf16x2(g23.x, g23.y);
         }
-        tmem_st16(tmem + lane_off + cS + c * 16, pp);
-        tmem_st16(tmem + lane_off + cDP + c * 16, pd);
-        // dS (query-major, 128-byte swizzle): this half's queries form block hf
+        // P^T and dS^T as bf16 pairs over the first 16 of this chunk's own 32 S^T / dP^T
+        // columns (never over columns the other warpgroup is still reading); the dV/dK
+        // MMAs read k-steps 0-1 of the half from chunk 0 and k-steps 2-3 from chunk 1
+        tmem_st16(tmem + lane_off + C::COL_S + q0, pp);
+        tmem_st16(tmem + lane_off + C::COL_DP + q0, pd);
+        // dS (query-major, 128-byte swizzle): half hf is block hf, this chunk units 4wg..4wg+3
         uint8_t* dsrow = smem + C::OFF_DS + (s % C::DS_BUF) * (128 * 128 * 2) + hf * (128 * 128) + r * 128;
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          const int unit = c * 4 + u;
+          const int unit = wg * 4 + u;
           *reinterpret_cast<uint4*>(dsrow + ((unit ^ (r & 7)) * 16)) =
               make_uint4(pd[4 * u], pd[4 * u + 1], pd[4 * u + 2], pd[4 * u + 3]);
         }
+        tmem_wait_st();
+        fence_proxy_async_smem();  // dS written by the generic proxy, read by the tensor core
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->ds_ready[hf]);
       }
-      tmem_wait_st();
-      fence_proxy_async_smem();  // dS written by the generic proxy, read by the tensor core
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->ds_ready[hf]);
     }
+    const int hf = wg;  // epilogue: warps 4-7 write dK, warps 8-11 dV
     // ---- dK_j (half A warps) and dV_j (half B warps); scale already folded into dS
     const uint32_t col = hf == 0 ? C::COL_DK : C::COL_DV;
     void* dst = hf == 0 ? p.dk : p.dv;
