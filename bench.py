@@ -369,6 +369,40 @@ def measure_decode(pc, dev, steps, warmup, world, peaks):
                                                                         "fa_paged_decode_combine_kernel"]}}
 
 
+def measure_append(pc, dev, steps, warmup, world, peaks):
+    """One new token per request written into the paged cache (KV-cache append)."""
+    import ctypes
+
+    import torch
+
+    import exact_attention_128_b200 as fa
+
+    inp = pc.make()
+    L = fa.lib()
+    kc, vc, table = inp["k_cache"].to(dev), inp["v_cache"].to(dev), inp["block_table"].to(dev)
+    # append at each request's last cached position (a slot its table already maps)
+    pos = (inp["ctx_lens"] - 1).to(torch.int32).to(dev)
+    k_new = torch.randn(pc.R, pc.Hkv, pc.d, device=dev).to(torch.bfloat16)
+    v_new = torch.randn(pc.R, pc.Hkv, pc.d, device=dev).to(torch.bfloat16)
+    args = [ctypes.c_void_p(t.data_ptr()) for t in (k_new, v_new, kc, vc, table, pos)]
+    args += [pc.R, pc.Hkv, pc.d, pc.block_size, pc.max_blocks_per_seq, inp["num_blocks"], fa.FA_DTYPE_BF16,
+             ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)]
+
+    def fn():
+        st = L.fa_paged_kv_append(*args)
+        if st != 0:
+            raise fa.FAError("fa_paged_kv_append", st)
+
+    ms = timed_loop([fn], steps, warmup, world)
+    per = ms / steps
+    nbytes = 2 * 2 * pc.R * pc.Hkv * pc.d * 2  # read the new K, V rows and write them
+    gbs = nbytes / (per * 1e-3) / 1e9
+    return {"per_step_ms": per, "gbs": gbs,
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 2), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(gbs / peaks["hbm_gbs"], 5), "algorithmic_bytes_per_step": nbytes,
+                         "note": "131 KB per call: launch-latency bound, not bandwidth bound"}}
+
+
 # ----------------------------------------------------------------------------- CPU oracle
 def oracle_threads():
     try:
@@ -459,7 +493,7 @@ def main():
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--only", choices=["prefill_causal", "prefill_noncausal", "train", "decode"],
+    ap.add_argument("--only", choices=["prefill_causal", "prefill_noncausal", "train", "decode", "append"],
                     help="measure just this one secondary workload (for profiling runs) and print it")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -493,6 +527,8 @@ def main():
             r = measure_train(W.TRAIN_CAUSAL, dev, args.steps, args.warmup, world, peaks)
         elif args.only == "decode":
             r = measure_decode(W.PAGED_DECODE, dev, args.steps, args.warmup, world, peaks)
+        elif args.only == "append":
+            r = measure_append(W.PAGED_DECODE, dev, args.steps, args.warmup, world, peaks)
         else:
             c = W.GQA_PREFILL_CAUSAL if args.only == "prefill_causal" else W.prefill_sweep()[3]
             r = measure_dense_fwd(c, dev, args.steps, args.warmup, world, peaks)
@@ -535,6 +571,10 @@ def main():
         r = measure_decode(W.PAGED_DECODE, dev, max(50, args.steps // 4), 10, world, peaks)
         secondary[W.PAGED_DECODE.name] = {"value": round(r["gbs"], 1), "unit": "GB/s",
                                           "ms_per_step": round(r["per_step_ms"], 5), "roofline": r["roofline"]}
+        r = measure_append(W.PAGED_DECODE, dev, max(50, args.steps // 4), 10, world, peaks)
+        secondary["paged_kv_append_r64_hkv2_d128"] = {"value": round(r["gbs"], 2), "unit": "GB/s",
+                                                      "ms_per_step": round(r["per_step_ms"], 5),
+                                                      "roofline": r["roofline"]}
 
     status = fa.device_status(reset=True)
     if status != 0:

@@ -25,6 +25,7 @@ __all__ = [
     "bwd_workspace_size",
     "paged_decode",
     "paged_decode_workspace_size",
+    "paged_kv_append",
     "device_status",
     "set_wait_limit_ns",
     "selftest_wait_timeout",
@@ -50,6 +51,7 @@ EXPORTED = {
     "fa_paged_decode_workspace_size": (_sz, [_i] * 5),
     "fa_paged_decode": (_i, [_vp] * 7 + [_i] * 7 + [_f, _i, _vp, _sz, _vp]),
     "fa_paged_decode_noalloc": (_i, [_vp] * 7 + [_i] * 7 + [_f, _i, _vp]),
+    "fa_paged_kv_append": (_i, [_vp] * 6 + [_i] * 6 + [_i, _vp]),
     "fa_device_status": (_i, [_i]),
     "fa_set_wait_limit_ns": (None, [ctypes.c_uint64]),
     "fa_selftest_wait_timeout": (_i, [_vp]),
@@ -191,6 +193,24 @@ def paged_decode(q, k_cache, v_cache, block_table, ctx_lens, scale: float | None
                                _stream())
     _check("fa_paged_decode", st)
     return o, lse
+
+
+def paged_kv_append(k_new, v_new, k_cache, v_cache, block_table, positions):
+    """Write one new token per request into the paged caches in place (slot positions[r])."""
+    _cuda4("k_new", k_new, torch.bfloat16)
+    _cuda4("v_new", v_new, torch.bfloat16)
+    _cuda4("k_cache", k_cache, torch.bfloat16)
+    _cuda4("v_cache", v_cache, torch.bfloat16)
+    _cuda4("block_table", block_table, torch.int32)
+    _cuda4("positions", positions, torch.int32)
+    if k_new.shape != v_new.shape or k_cache.shape != v_cache.shape:
+        raise ValueError("k/v shapes disagree")
+    R, Hkv, d = k_new.shape
+    num_blocks, _, bs, _ = k_cache.shape
+    st = lib().fa_paged_kv_append(_ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
+                                  _ptr(positions), R, Hkv, d, bs, block_table.shape[1], num_blocks, FA_DTYPE_BF16,
+                                  _stream())
+    _check("fa_paged_kv_append", st)
 
 
 def device_status(reset: bool = True) -> int:

@@ -317,6 +317,33 @@ __global__ void __launch_bounds__(dec::WARPS * 32)
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// Append one token per request: thread group (r, h) copies the 256-byte key and value
+// rows of the new token into slot pos % 16 of physical block block_table[r][pos / 16].
+__global__ void __launch_bounds__(128) fa_paged_kv_append_kernel(const uint4* k_new, const uint4* v_new, uint4* kc,
+                                                                 uint4* vc, const int* bt, const int* pos, int R,
+                                                                 int Hkv, int max_blocks, int num_blocks) {
+  using namespace dec;
+  constexpr int PER_ROW = D * 2 / 16;  // 16-byte pieces per 256-byte row
+  const long gid = long(blockIdx.x) * blockDim.x + threadIdx.x;
+  const long rh = gid / PER_ROW;
+  const int piece = int(gid % PER_ROW);
+  if (rh >= long(R) * Hkv) return;
+  const int r = int(rh / Hkv), h = int(rh % Hkv);
+  const int t = pos[r];
+  if (t < 0 || t >= max_blocks * BS) {
+    if (piece == 0) set_status(FA_ERR_INVALID_ARG, 110);
+    return;
+  }
+  const int phys = bt[size_t(r) * max_blocks + t / BS];
+  if (phys < 0 || phys >= num_blocks) {
+    if (piece == 0) set_status(FA_ERR_INVALID_ARG, 111);
+    return;
+  }
+  const size_t dst = ((size_t(phys) * Hkv + h) * BS + t % BS) * PER_ROW + piece;
+  kc[dst] = k_new[rh * PER_ROW + piece];
+  vc[dst] = v_new[rh * PER_ROW + piece];
+}
+
 // Merge the split partials of requests that needed more than one split: each split's
 // normalised output is weighted by e^{lse_s - lse}, lse = ln sum_s e^{lse_s}.
 __global__ void __launch_bounds__(128) fa_paged_decode_combine_kernel(const DecodeParams p) {

@@ -310,6 +310,23 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                     static_cast<cudaStream_t>(stream));
 }
 
+fa_status fa_paged_kv_append(const void* k_new, const void* v_new, void* k_cache, void* v_cache,
+                             const int* block_table, const int* positions, int R, int Hkv, int d, int block_size,
+                             int max_blocks_per_seq, int num_blocks, fa_dtype dtype, void* stream) {
+  if (!k_new || !v_new || !k_cache || !v_cache || !block_table || !positions) return FA_ERR_INVALID_ARG;
+  if (R <= 0 || Hkv <= 0 || d <= 0 || block_size <= 0 || max_blocks_per_seq <= 0 || num_blocks <= 0)
+    return FA_ERR_INVALID_ARG;
+  if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+      !aligned(block_table, 4) || !aligned(positions, 4))
+    return FA_ERR_INVALID_ARG;
+  if (dtype != FA_DTYPE_BF16 || d != dec::D || block_size != dec::BS) return FA_ERR_UNSUPPORTED;
+  const long threads = long(R) * Hkv * (dec::D * 2 / 16);
+  fa_paged_kv_append_kernel<<<int((threads + 127) / 128), 128, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new), static_cast<uint4*>(k_cache),
+      static_cast<uint4*>(v_cache), block_table, positions, R, Hkv, max_blocks_per_seq, num_blocks);
+  return launched();
+}
+
 size_t fa_paged_decode_workspace_size(int R, int Hq, int d, int max_blocks_per_seq, int block_size) {
   if (R <= 0 || Hq <= 0 || d <= 0 || max_blocks_per_seq <= 0 || block_size <= 0) return 0;
   const size_t splits = size_t((max_blocks_per_seq + dec::CHUNK - 1) / dec::CHUNK);

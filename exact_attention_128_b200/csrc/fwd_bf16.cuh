@@ -41,6 +41,12 @@ namespace fa {
 #define FWD_EMU_PAIRS 0x00u
 #endif
 
+// Lazy rescaling threshold (base-2 units) for the running reference maximum; see the
+// softmax loop.  8 keeps every P <= 256, far inside bf16 and fp32 range.
+#ifndef FA_RESCALE_LOG2
+#define FA_RESCALE_LOG2 8.0f
+#endif
+
 // Two configurations:
 //   BN = 128 (d = 128): 384 threads (softmax warps 4-11), 512 TMEM columns, one CTA/SM.
 //   BN = 64  (d = 64):  320 threads (softmax warps 2-9), 256 TMEM columns and ~97 KB of
@@ -294,14 +300,19 @@ __global__ void __launch_bounds__(FwdCfg<D, BN>::THREADS, FwdCfg<D, BN>::CTAS_PE
           }
           float mx8[8];
 #pragma unroll
-          for (int k = 0; k < 8; ++k) mx8[k] = f[k];
+          for (int k = 0; k < 8; ++k) mx8[k] = fmaxf(f[k], f[8 + k]);
 #pragma unroll
-          for (int c = 8; c < C::BN; c += 8)
+          for (int c = 16; c < C::BN; c += 16)
 #pragma unroll
-            for (int k = 0; k < 8; ++k) mx8[k] = fmaxf(mx8[k], f[c + k]);
-          const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                 fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-          const float m_new = fmaxf(m, mx * sl2);
+            for (int k = 0; k < 8; ++k) mx8[k] = fmax3(mx8[k], f[c + k], f[c + 8 + k]);
+          const float mx = fmaxf(fmax3(mx8[0], mx8[1], mx8[2]),
+                                 fmaxf(fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+          // The reference m that l and u share moves only when the row maximum exceeds it
+          // by more than FA_RESCALE_LOG2 (base 2): u / l does not depend on which reference
+          // they share, and until then every P = 2^(s - m) stays below 2^FA_RESCALE_LOG2.
+          // With FA_RESCALE_LOG2 = 0 this is the recurrence with m the exact running max.
+          const float m_cand = fmaxf(m, mx * sl2);
+          const float m_new = (m_cand > m + FA_RESCALE_LOG2) ? m_cand : m;
           const float base = (m_new == -INFINITY) ? 0.f : m_new;
           const float alpha = (m_new == m) ? 1.f : ex2(m - base);
           const float2 sl2v = make_float2(sl2, sl2), nbase = make_float2(-base, -base);

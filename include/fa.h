@@ -132,6 +132,26 @@ fa_status fa_paged_decode(const void* q, const void* k_cache, const void* v_cach
                           void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * fa_paged_kv_append — writes one new token per request into a paged KV cache ("Atención
+ * tipo FlashAttention y atención paginada": the cache grows one token at a time and the
+ * block table links logical positions to fixed-size physical blocks).
+ *   k_new, v_new [R, Hkv, d] bf16: the new token's key and value for every KV head.
+ *   positions [R] int32 (device): logical position of the new token in request r
+ *     (its context length before the append); it goes to physical block
+ *     block_table[r][pos / block_size], slot pos % block_size.
+ *   k_cache, v_cache [num_blocks, Hkv, block_size, d] bf16, updated in place;
+ *   block_table [R, max_blocks_per_seq] int32.
+ *   d == 128, block_size == 16.  A position outside [0, max_blocks_per_seq*block_size)
+ *   or a physical block outside [0, num_blocks) is not written; the kernel sets the
+ *   device status word (FA_ERR_INVALID_ARG) instead.
+ * Errors: FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED.
+ */
+fa_status fa_paged_kv_append(const void* k_new, const void* v_new, void* k_cache, void* v_cache,
+                             const int* block_table, const int* positions, int R, int Hkv, int d,
+                             int block_size, int max_blocks_per_seq, int num_blocks, fa_dtype dtype,
+                             void* stream);
+
+/*
  * fa_paged_decode_noalloc — fa_paged_decode for callers that cannot allocate device
  * memory.  (No counterpart on the pages: this is a deployment variant of the decode
  * step, not part of the method.)

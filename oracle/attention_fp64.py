@@ -44,6 +44,7 @@ __all__ = [
     "paged_decode",
     "online_softmax_blocks",
     "merge_partials",
+    "paged_append",
 ]
 
 
@@ -277,3 +278,19 @@ def merge_partials(lse_parts, o_parts):
     lse = top + np.log(w.sum())
     O = (w[:, None] * o_parts.reshape(len(lse_parts), -1)).sum(axis=0) / w.sum()
     return O.reshape(o_parts.shape[1:]), lse
+
+
+def paged_append(k_cache, v_cache, block_table, positions, k_new, v_new, block_size: int):
+    """The caches after appending one token per request ([KR] "Atención tipo FlashAttention
+    y atención paginada": the cache grows one token at a time; the block table links the
+    logical position to a physical block).  Request r's new key/value for every KV head
+    goes to block ``block_table[r][pos // block_size]``, slot ``pos % block_size``.  Works
+    on copies of the stored values (no arithmetic); returns (k_cache, v_cache)."""
+    kc = np.array(k_cache, copy=True)
+    vc = np.array(v_cache, copy=True)
+    table = np.asarray(block_table)
+    for r, pos in enumerate(np.asarray(positions)):
+        pb = int(table[r, int(pos) // block_size])
+        kc[pb, :, int(pos) % block_size] = np.asarray(k_new)[r]
+        vc[pb, :, int(pos) % block_size] = np.asarray(v_new)[r]
+    return kc, vc

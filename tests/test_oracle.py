@@ -389,3 +389,27 @@ def test_planted_mistakes_are_caught(monkeypatch):
         assert not _pins_pass(), label
         monkeypatch.undo()
     assert _pins_pass()
+
+
+def test_paged_append_token_by_token_rebuilds_the_sequence():
+    """Appending a sequence one token at a time into an empty paged cache, then de-paging,
+    gives back the sequence (the cache grows one token at a time through the table)."""
+    rng = np.random.default_rng(18)
+    Hkv, d, bs, n = 2, 3, 4, 13
+    seq_k = rng.standard_normal((n, Hkv, d))
+    seq_v = rng.standard_normal((n, Hkv, d))
+    nblk = (n + bs - 1) // bs
+    table = np.full((1, nblk + 1), -1)
+    table[0, :nblk] = rng.permutation(10)[:nblk]
+    kc = np.zeros((10, Hkv, bs, d))
+    vc = np.zeros((10, Hkv, bs, d))
+    for t in range(n):
+        kc, vc = ora.paged_append(kc, vc, table, [t], seq_k[t][None], seq_v[t][None], bs)
+    for g in range(Hkv):
+        np.testing.assert_array_equal(ora.depage(kc, table[0], n, g, bs), seq_k[:, g])
+        np.testing.assert_array_equal(ora.depage(vc, table[0], n, g, bs), seq_v[:, g])
+    # untouched blocks stay untouched
+    used = set(int(x) for x in table[0, :nblk])
+    for b in range(10):
+        if b not in used:
+            assert not kc[b].any()
