@@ -91,7 +91,7 @@ class ClockSampler:
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=self.fh, stderr=subprocess.DEVNULL)
+                 "-lms", "20"], stdout=self.fh, stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
         self.t0 = time.time()
@@ -486,7 +486,7 @@ def reference_line(case, args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--steps", type=int, default=10000)
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="vit_b16_batched_fwd_bf16")
@@ -557,21 +557,21 @@ def main():
         for c in (W.GQA_PREFILL_CAUSAL, W.prefill_sweep()[3]):
             if c.name == case.name:
                 continue
-            r = measure_dense_fwd(c, dev, max(20, args.steps // 50), 5, world, peaks)
+            r = measure_dense_fwd(c, dev, 20, 5, world, peaks)
             secondary[c.name] = {"value": round(r["tflops"], 2), "unit": "TFLOP/s",
                                  "ms_per_step": round(r["per_step_ms"], 4), "roofline": r["roofline"]}
             torch.cuda.empty_cache()
         try:
-            r = measure_train(W.TRAIN_CAUSAL, dev, max(10, args.steps // 100), 3, world, peaks)
+            r = measure_train(W.TRAIN_CAUSAL, dev, 10, 3, world, peaks)
             secondary[W.TRAIN_CAUSAL.name] = {"value": round(r["tflops"], 2), "unit": "TFLOP/s",
                                               "ms_per_step": round(r["per_step_ms"], 4), "roofline": r["roofline"]}
         except fa.FAError as e:
             secondary[W.TRAIN_CAUSAL.name] = {"unavailable": str(e)}
         torch.cuda.empty_cache()
-        r = measure_decode(W.PAGED_DECODE, dev, max(50, args.steps // 4), 10, world, peaks)
+        r = measure_decode(W.PAGED_DECODE, dev, 300, 10, world, peaks)
         secondary[W.PAGED_DECODE.name] = {"value": round(r["gbs"], 1), "unit": "GB/s",
                                           "ms_per_step": round(r["per_step_ms"], 5), "roofline": r["roofline"]}
-        r = measure_append(W.PAGED_DECODE, dev, max(50, args.steps // 4), 10, world, peaks)
+        r = measure_append(W.PAGED_DECODE, dev, 300, 10, world, peaks)
         secondary["paged_kv_append_r64_hkv2_d128"] = {"value": round(r["gbs"], 2), "unit": "GB/s",
                                                       "ms_per_step": round(r["per_step_ms"], 5),
                                                       "roofline": r["roofline"]}

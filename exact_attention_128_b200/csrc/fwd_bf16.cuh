@@ -8,9 +8,9 @@
 // a tile raises the maximum, l and u are rescaled by e^{m - m'} before the tile's own
 // terms are added; the output is u / l.
 //
-// Persistent kernel: one CTA per SM walks work items (two 128-row query tiles Q0, Q1 of
-// one (batch, query head)), item = blockIdx.x + k * gridDim.x; causal items are ordered
-// heaviest first.  Each item streams the 128-key tiles of its key/value head (GQA: head
+// Persistent kernel: CTAs walk work items (two 128-row query tiles Q0, Q1 of one (batch,
+// query head)), item = blockIdx.x + k * gridDim.x, ordered head-major (non-causal: K/V
+// reuse in L2) or longest-first (causal).  Each item streams the 128-key tiles of its key/value head (GQA: head
 // h reads h / (Hq/Hkv)).  The K/V ring and the Q buffers run ahead across item
 // boundaries, so loads for the next item overlap the current item's tail and epilogue.
 //   warp 0      TMA producer: Q0/Q1 per item (QBUF buffers), K_j and V_j into a ring.
@@ -112,9 +112,13 @@ __global__ void __launch_bounds__(FwdCfg<D, BN>::THREADS, FwdCfg<D, BN>::CTAS_PE
   const int n_qp = (p.Nq + 2 * C::BM - 1) / (2 * C::BM);
   const int n_items = n_qp * p.BH;
   const int off = p.Nkv - p.Nq;  // bottom-right causal alignment
-  // item -> (query-tile pair, batch*head); causal items heaviest (last query tiles) first
-  auto item_qt = [&](int it) { return CAUSAL ? n_qp - 1 - it / p.BH : it / p.BH; };
-  auto item_bh = [&](int it) { return it % p.BH; };
+  // item -> (query-tile pair, batch*head).  Non-causal items are head-major, so the CTAs
+  // running at the same time share one or two heads' K/V in L2 (at N = 8192 this cut
+  // DRAM traffic per launch from 4.2 GB to the 0.64 GB of the algorithm); causal items are
+  // longest-first over all heads (last query tiles first), which balances their very
+  // unequal lengths better than any head grouping measured.
+  auto item_qt = [&](int it) { return CAUSAL ? n_qp - 1 - it / p.BH : it % n_qp; };
+  auto item_bh = [&](int it) { return CAUSAL ? it % p.BH : it / n_qp; };
   auto item_ntiles = [&](int qt) {
     int kv_end = p.Nkv;
     if (CAUSAL) kv_end = min(p.Nkv, min(qt * 2 * C::BM + 2 * C::BM, p.Nq) + off);
