@@ -403,6 +403,45 @@ def measure_append(pc, dev, steps, warmup, world, peaks):
                          "note": "131 KB per call: launch-latency bound, not bandwidth bound"}}
 
 
+def measure_graph_decode(dev, steps, warmup, world):
+    """A small, launch-bound decode step (8 requests, append + decode) issued eagerly
+    through the C ABI vs replayed from a CUDA graph; per-step device time of each."""
+    import torch
+
+    import exact_attention_128_b200 as fa
+    from exact_attention_128_b200.workloads import PagedCase
+
+    pc = PagedCase("graph_decode_r8", 8, 12, 2, 128, 16, 512, 1024, 64, 71)
+    inp = pc.make()
+    kc, vc, table = inp["k_cache"].to(dev), inp["v_cache"].to(dev), inp["block_table"].to(dev)
+    q = inp["q"].to(dev)
+    ctx = inp["ctx_lens"].to(dev)
+    pos = (inp["ctx_lens"] - 1).to(dev)
+    k_new = torch.randn(pc.R, pc.Hkv, pc.d, device=dev).to(torch.bfloat16)
+    v_new = torch.randn_like(k_new)
+    o = torch.empty_like(q)
+    ws = torch.empty(fa.paged_decode_workspace_size(pc.R, pc.Hq, pc.d, pc.max_blocks_per_seq, pc.block_size),
+                     device=dev, dtype=torch.uint8)
+
+    def step():
+        fa.paged_kv_append(k_new, v_new, kc, vc, table, pos)
+        fa.paged_decode(q, kc, vc, table, ctx, with_lse=False, workspace=ws, out=o)
+
+    eager = timed_loop([step], steps, warmup, world) / steps
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        step()
+    torch.cuda.current_stream().wait_stream(s)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
+    graph = timed_loop([g.replay], steps, warmup, world) / steps
+    del g
+    return {"eager_ms_per_step": round(eager, 5), "graph_ms_per_step": round(graph, 5),
+            "speedup": round(eager / graph, 3), "kernels_per_step": 3}
+
+
 # ----------------------------------------------------------------------------- CPU oracle
 def oracle_threads():
     try:
@@ -493,7 +532,7 @@ def main():
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--only", choices=["prefill_causal", "prefill_noncausal", "train", "decode", "append"],
+    ap.add_argument("--only", choices=["prefill_causal", "prefill_noncausal", "train", "decode", "append", "graph"],
                     help="measure just this one secondary workload (for profiling runs) and print it")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -529,6 +568,8 @@ def main():
             r = measure_decode(W.PAGED_DECODE, dev, args.steps, args.warmup, world, peaks)
         elif args.only == "append":
             r = measure_append(W.PAGED_DECODE, dev, args.steps, args.warmup, world, peaks)
+        elif args.only == "graph":
+            r = measure_graph_decode(dev, args.steps, args.warmup, world)
         else:
             c = W.GQA_PREFILL_CAUSAL if args.only == "prefill_causal" else W.prefill_sweep()[3]
             r = measure_dense_fwd(c, dev, args.steps, args.warmup, world, peaks)
@@ -571,6 +612,7 @@ def main():
         r = measure_decode(W.PAGED_DECODE, dev, 300, 10, world, peaks)
         secondary[W.PAGED_DECODE.name] = {"value": round(r["gbs"], 1), "unit": "GB/s",
                                           "ms_per_step": round(r["per_step_ms"], 5), "roofline": r["roofline"]}
+        secondary["graph_decode_r8_append_plus_decode"] = measure_graph_decode(dev, 300, 10, world)
         r = measure_append(W.PAGED_DECODE, dev, 300, 10, world, peaks)
         secondary["paged_kv_append_r64_hkv2_d128"] = {"value": round(r["gbs"], 2), "unit": "GB/s",
                                                       "ms_per_step": round(r["per_step_ms"], 5),
