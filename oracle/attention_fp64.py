@@ -45,6 +45,7 @@ __all__ = [
     "online_softmax_blocks",
     "merge_partials",
     "paged_append",
+    "paged_prefill",
 ]
 
 
@@ -294,3 +295,32 @@ def paged_append(k_cache, v_cache, block_table, positions, k_new, v_new, block_s
         kc[pb, :, int(pos) % block_size] = np.asarray(k_new)[r]
         vc[pb, :, int(pos) % block_size] = np.asarray(v_new)[r]
     return kc, vc
+
+
+def paged_prefill(q, k_cache, v_cache, block_table, ctx_lens, q_lens, block_size: int, scale: float,
+                  causal: bool):
+    """Prefill over a paged KV cache -> (O [R,Hq,Nq_max,d], lse [R,Hq,Nq_max]).
+
+    [KR] "Atención tipo FlashAttention y atención paginada" joins blockwise prefill with
+    the paged cache.  Request r has ``ctx_lens[r]`` cached tokens (de-paged through its
+    block-table row) and ``q_lens[r]`` query rows, which are the last ``q_lens[r]``
+    positions of its sequence (bottom-right causal alignment).  Rows at and past
+    ``q_lens[r]`` are left as NaN: they are not part of the result.
+    """
+    q = to_f64(q)
+    k_cache, v_cache = to_f64(k_cache), to_f64(v_cache)
+    table = np.asarray(block_table)
+    R, Hq, Nq_max, d = q.shape
+    G = _check_gqa(Hq, k_cache.shape[1])
+    O = np.full((R, Hq, Nq_max, v_cache.shape[-1]), np.nan)
+    lse = np.full((R, Hq, Nq_max), np.nan)
+    for r in range(R):
+        n, nq = int(np.asarray(ctx_lens)[r]), int(np.asarray(q_lens)[r])
+        if not (1 <= nq <= n):
+            raise ValueError("need 1 <= q_len <= ctx_len")
+        for g in range(k_cache.shape[1]):
+            kr = depage(k_cache, table[r], n, g, block_size)
+            vr = depage(v_cache, table[r], n, g, block_size)
+            for h in range(g * G, (g + 1) * G):
+                O[r, h, :nq], lse[r, h, :nq], _ = attention_head(q[r, h, :nq], kr, vr, scale, causal)
+    return O, lse

@@ -413,3 +413,31 @@ def test_paged_append_token_by_token_rebuilds_the_sequence():
     for b in range(10):
         if b not in used:
             assert not kc[b].any()
+
+
+def test_paged_prefill_equals_dense_and_decode():
+    """Full prefill from pages equals dense attention on the contiguous K/V; a one-row
+    prefill equals the decode step; rows past q_len are not part of the result."""
+    rng = np.random.default_rng(19)
+    R, Hq, Hkv, d, bs = 3, 4, 2, 3, 4
+    ctx = [1, 9, 13]
+    ks = [rng.standard_normal((Hkv, n, d)) for n in ctx]
+    vs = [rng.standard_normal((Hkv, n, d)) for n in ctx]
+    kc, table = _scatter_to_pages(ks, bs, Hkv, d, np.random.default_rng(3))
+    vc, _ = _scatter_to_pages(vs, bs, Hkv, d, np.random.default_rng(3))
+    nq_max = 13
+    q = rng.standard_normal((R, Hq, nq_max, d))
+    for causal in (False, True):
+        O, L = ora.paged_prefill(q, kc, vc, table, ctx, ctx, bs, 0.5, causal)  # q_len = ctx
+        for r in range(R):
+            Od, Ld = ora.attention_fwd(q[r:r + 1, :, :ctx[r]], ks[r][None], vs[r][None], 0.5, causal)
+            np.testing.assert_allclose(O[r, :, :ctx[r]], Od[0], atol=1e-14)
+            np.testing.assert_allclose(L[r, :, :ctx[r]], Ld[0], atol=1e-14)
+            assert np.isnan(O[r, :, ctx[r]:]).all()
+    # one query row at the end of each sequence is the decode step (causal or not)
+    O1, L1 = ora.paged_prefill(q, kc, vc, table, ctx, [1, 1, 1], bs, 0.5, True)
+    Od, Ldd = ora.paged_decode(q[:, :, 0], kc, vc, table, ctx, bs, 0.5)
+    np.testing.assert_allclose(O1[:, :, 0], Od, atol=1e-14)
+    np.testing.assert_allclose(L1[:, :, 0], Ldd, atol=1e-14)
+    with pytest.raises(ValueError):
+        ora.paged_prefill(q, kc, vc, table, ctx, [2, 10, 3], bs, 0.5, True)
