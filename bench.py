@@ -369,6 +369,53 @@ def measure_decode(pc, dev, steps, warmup, world, peaks):
                                                                         "fa_paged_decode_combine_kernel"]}}
 
 
+def measure_paged_prefill(pc, dev, steps, warmup, world, peaks, peak_key="bf16_tflops"):
+    """Prefill over the paged cache: 4*d FLOP per computed (query, key) pair and head;
+    bytes = every cached K/V row once per KV head + q and o rows (bf16)."""
+    import ctypes
+
+    import torch
+
+    import exact_attention_128_b200 as fa
+
+    inp = pc.make()
+    names = ("q", "k_cache", "v_cache", "block_table", "ctx_lens", "q_lens")
+    set_bytes = (inp["k_cache"].numel() * 2 + inp["q"].numel() * 2) * 2
+    rot = n_rotations(set_bytes)
+    L = fa.lib()
+    base = {n: inp[n].to(dev) for n in names}
+    R, Hq, nq_max, d = inp["q"].shape
+    fns, keep = [], []
+    for i in range(rot):
+        s = base if i == 0 else {n: t.clone() for n, t in base.items()}
+        o = torch.empty_like(s["q"])
+        lse = torch.empty(R, Hq, nq_max, device=dev, dtype=torch.float32)
+        keep.append((s, o, lse))
+        args = [ctypes.c_void_p(s[n].data_ptr()) for n in names]
+        args += [ctypes.c_void_p(o.data_ptr()), ctypes.c_void_p(lse.data_ptr()), R, Hq, pc.Hkv, nq_max, d,
+                 pc.block_size, pc.max_blocks_per_seq, inp["num_blocks"], ctypes.c_float(pc.scale), int(pc.causal),
+                 fa.FA_DTYPE_BF16, ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)]
+
+        def fn(args=args):
+            st = L.fa_paged_prefill(*args)
+            if st != 0:
+                raise fa.FAError("fa_paged_prefill", st)
+
+        fns.append(fn)
+    ms = timed_loop(fns, steps, warmup, world)
+    per = ms / steps
+    flops = pc.fwd_flops()
+    tflops = flops / (per * 1e-3) / 1e12
+    peak = peaks[peak_key]
+    kname = f"fa_fwd_bf16_kernel<{pc.d},{str(pc.causal).lower()},paged>"
+    return {"per_step_ms": per, "tflops": tflops,
+            "roofline": {"bound": "tensor", "achieved": round(tflops, 2), "peak": peak, "unit": "TFLOP/s",
+                         "frac": round(tflops / peak, 4), "peak_kind": peak_key,
+                         "frac_of_nominal_2250": round(tflops / NOMINAL_BF16_TFLOPS, 4),
+                         "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": pc.io_bytes(),
+                         "kernel": kname, "traffic": traffic_for(kname)}}
+
+
 def measure_append(pc, dev, steps, warmup, world, peaks):
     """One new token per request written into the paged cache (KV-cache append)."""
     import ctypes
@@ -532,7 +579,8 @@ def main():
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--only", choices=["prefill_causal", "prefill_noncausal", "train", "decode", "append", "graph"],
+    ap.add_argument("--only", choices=["prefill_causal", "prefill_noncausal", "train", "decode", "append", "graph",
+                                       "paged_prefill"],
                     help="measure just this one secondary workload (for profiling runs) and print it")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -570,6 +618,8 @@ def main():
             r = measure_append(W.PAGED_DECODE, dev, args.steps, args.warmup, world, peaks)
         elif args.only == "graph":
             r = measure_graph_decode(dev, args.steps, args.warmup, world)
+        elif args.only == "paged_prefill":
+            r = measure_paged_prefill(W.PAGED_PREFILL, dev, args.steps, args.warmup, world, peaks)
         else:
             c = W.GQA_PREFILL_CAUSAL if args.only == "prefill_causal" else W.prefill_sweep()[3]
             r = measure_dense_fwd(c, dev, args.steps, args.warmup, world, peaks)
@@ -608,6 +658,10 @@ def main():
                                               "ms_per_step": round(r["per_step_ms"], 4), "roofline": r["roofline"]}
         except fa.FAError as e:
             secondary[W.TRAIN_CAUSAL.name] = {"unavailable": str(e)}
+        torch.cuda.empty_cache()
+        r = measure_paged_prefill(W.PAGED_PREFILL, dev, 20, 5, world, peaks)
+        secondary[W.PAGED_PREFILL.name] = {"value": round(r["tflops"], 2), "unit": "TFLOP/s",
+                                           "ms_per_step": round(r["per_step_ms"], 4), "roofline": r["roofline"]}
         torch.cuda.empty_cache()
         r = measure_decode(W.PAGED_DECODE, dev, 300, 10, world, peaks)
         secondary[W.PAGED_DECODE.name] = {"value": round(r["gbs"], 1), "unit": "GB/s",

@@ -26,6 +26,7 @@ __all__ = [
     "paged_decode",
     "paged_decode_workspace_size",
     "paged_kv_append",
+    "paged_prefill",
     "device_status",
     "set_wait_limit_ns",
     "selftest_wait_timeout",
@@ -52,6 +53,7 @@ EXPORTED = {
     "fa_paged_decode": (_i, [_vp] * 7 + [_i] * 7 + [_f, _i, _vp, _sz, _vp]),
     "fa_paged_decode_noalloc": (_i, [_vp] * 7 + [_i] * 7 + [_f, _i, _vp]),
     "fa_paged_kv_append": (_i, [_vp] * 6 + [_i] * 6 + [_i, _vp]),
+    "fa_paged_prefill": (_i, [_vp] * 6 + [_vp, _vp] + [_i] * 8 + [_f, _i, _i, _vp]),
     "fa_device_status": (_i, [_i]),
     "fa_set_wait_limit_ns": (None, [ctypes.c_uint64]),
     "fa_selftest_wait_timeout": (_i, [_vp]),
@@ -211,6 +213,33 @@ def paged_kv_append(k_new, v_new, k_cache, v_cache, block_table, positions):
                                   _ptr(positions), R, Hkv, d, bs, block_table.shape[1], num_blocks, FA_DTYPE_BF16,
                                   _stream())
     _check("fa_paged_kv_append", st)
+
+
+def paged_prefill(q, k_cache, v_cache, block_table, ctx_lens, q_lens, causal: bool = True,
+                  scale: float | None = None, out=None, lse=None):
+    """Prefill over a paged KV cache: q [R,Hq,Nq_max,d] (request r's rows < q_lens[r] are its
+    last q_lens[r] positions), caches [num_blocks,Hkv,block_size,d] -> (o, lse [R,Hq,Nq_max]).
+    Rows >= q_lens[r] of o and lse are undefined."""
+    _cuda4("q", q, torch.bfloat16)
+    _cuda4("k_cache", k_cache, torch.bfloat16)
+    _cuda4("v_cache", v_cache, torch.bfloat16)
+    _cuda4("block_table", block_table, torch.int32)
+    _cuda4("ctx_lens", ctx_lens, torch.int32)
+    _cuda4("q_lens", q_lens, torch.int32)
+    if q.dim() != 4 or k_cache.dim() != 4 or v_cache.shape != k_cache.shape:
+        raise ValueError("expected q [R,Hq,Nq_max,d] and caches [num_blocks,Hkv,block_size,d]")
+    R, Hq, Nq, d = q.shape
+    num_blocks, Hkv, bs, _ = k_cache.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    o = out if out is not None else torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((R, Hq, Nq), device=q.device, dtype=torch.float32)
+    st = lib().fa_paged_prefill(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(ctx_lens),
+                                _ptr(q_lens), _ptr(o), _ptr(lse), R, Hq, Hkv, Nq, d, bs, block_table.shape[1],
+                                num_blocks, float(scale), int(bool(causal)), FA_DTYPE_BF16, _stream())
+    _check("fa_paged_prefill", st)
+    return o, lse
 
 
 def device_status(reset: bool = True) -> int:

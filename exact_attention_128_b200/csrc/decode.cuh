@@ -10,7 +10,7 @@
 // ("Mecanismo y detalles", GQA) are processed together, so each K/V byte is read once.
 //
 // Work split (split-KV): CTA (split s, kv head g, request r) covers logical blocks
-// [s*CHUNK, (s+1)*CHUNK) of request r (CHUNK = 64 blocks = 1024 tokens by default).  Each
+// [s*CHUNK, (s+1)*CHUNK) of request r (CHUNK = 128 blocks = 2048 tokens by default).  Each
 // of its 4 warps takes every 4th block and
 // keeps its own (m, l, u) state; the warps' states and then the splits' partial
 // results are merged by weighting each part with its unnormalised mass e^{lse_s}
@@ -31,10 +31,10 @@ namespace dec {
 constexpr int D = 128;
 constexpr int BS = 16;          // tokens per cache block
 #ifndef FA_DEC_STAGES
-#define FA_DEC_STAGES 3
+#define FA_DEC_STAGES 2
 #endif
 #ifndef FA_DEC_CHUNK
-#define FA_DEC_CHUNK 64
+#define FA_DEC_CHUNK 128
 #endif
 constexpr int WARPS = 4;
 constexpr int STAGES = FA_DEC_STAGES;  // blocks in flight per warp
@@ -80,14 +80,6 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t&
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
                : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
                : "r"(addr));
-}
-
-__device__ __forceinline__ void tma_load_2d(uint32_t smem_dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
-      "[%2];" ::"r"(smem_dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
-      : "memory");
 }
 
 // Byte offset of 16-byte chunk `chunk` (0..15) of slab row `row` (0..15) in a stage

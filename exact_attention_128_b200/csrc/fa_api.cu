@@ -55,13 +55,13 @@ bool make_map_bf16(CUtensorMap* m, const void* base, int d, int rows, int planes
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// 2-D bf16 map over a paged cache viewed as [rows][128] with a (64, 16) box and the
-// 128-byte swizzle: one box is half of one (block, kv head) slab.
-bool make_map_cache(CUtensorMap* m, const void* base, long rows) {
+// 2-D bf16 map over a paged cache viewed as [rows][d] with a (64, 16) box and the
+// 128-byte swizzle: one box is one 64-column block of one (block, kv head) slab.
+bool make_map_cache(CUtensorMap* m, const void* base, long rows, int d = 128) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
-  cuuint64_t dims[2] = {128, cuuint64_t(rows)};
-  cuuint64_t strides[1] = {256};
+  cuuint64_t dims[2] = {cuuint64_t(d), cuuint64_t(rows)};
+  cuuint64_t strides[1] = {cuuint64_t(d) * 2};
   cuuint32_t box[2] = {64, 16};
   cuuint32_t estr[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
@@ -84,11 +84,11 @@ int sm_count() {
   return n;
 }
 
-template <int D, int BN, bool CAUSAL>
+template <int D, int BN, bool CAUSAL, bool PAGED = false>
 fa_status launch_fwd_bf16(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                           const CUtensorMap& mo, const FwdBf16Params& prm, int Nq, cudaStream_t st) {
   using C = FwdCfg<D, BN>;
-  auto kern = fa_fwd_bf16_kernel<D, BN, CAUSAL>;
+  auto kern = fa_fwd_bf16_kernel<D, BN, CAUSAL, PAGED>;
   if (set_smem(kern, C::SMEM) != cudaSuccess) return FA_ERR_CUDA;
   const long items = long((Nq + 2 * C::BM - 1) / (2 * C::BM)) * prm.BH;
   const long slots = long(sm_count()) * C::CTAS_PER_SM;
@@ -272,12 +272,46 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
       !make_map_bf16(&mv, v, d, Nkv, B * Hkv, bn) || !make_map_bf16(&mo, o, d, Nq, B * Hq, 32))
     return FA_ERR_CUDA;
   FwdBf16Params prm{static_cast<__nv_bfloat16*>(o), lse, B * Hq, Hq, Hkv, Nq, Nkv,
-                    scale * 1.4426950408889634f, g_wait_ns};
+                    scale * 1.4426950408889634f, g_wait_ns, nullptr, nullptr, nullptr, 0, 0};
   if (d == 64)
     return causal ? launch_fwd_bf16<64, BN64, true>(mq, mk, mv, mo, prm, Nq, st)
                   : launch_fwd_bf16<64, BN64, false>(mq, mk, mv, mo, prm, Nq, st);
   return causal ? launch_fwd_bf16<128, 128, true>(mq, mk, mv, mo, prm, Nq, st)
                 : launch_fwd_bf16<128, 128, false>(mq, mk, mv, mo, prm, Nq, st);
+}
+
+fa_status fa_paged_prefill(const void* q, const void* k_cache, const void* v_cache, const int* block_table,
+                           const int* ctx_lens, const int* q_lens, void* o, float* lse, int R, int Hq, int Hkv,
+                           int Nq_max, int d, int block_size, int max_blocks_per_seq, int num_blocks, float scale,
+                           int causal, fa_dtype dtype, void* stream) {
+  if (!q || !k_cache || !v_cache || !block_table || !ctx_lens || !q_lens || !o || !lse) return FA_ERR_INVALID_ARG;
+  if (R <= 0 || Hq <= 0 || Hkv <= 0 || Nq_max <= 0 || d <= 0 || block_size <= 0 || max_blocks_per_seq <= 0 ||
+      num_blocks <= 0)
+    return FA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(o, 16) || !aligned(lse, 4) ||
+      !aligned(block_table, 4) || !aligned(ctx_lens, 4) || !aligned(q_lens, 4))
+    return FA_ERR_INVALID_ARG;
+  if (dtype != FA_DTYPE_BF16 || (d != 64 && d != 128) || block_size != 16) return FA_ERR_UNSUPPORTED;
+  if (long(R) * Hq > 65535) return FA_ERR_UNSUPPORTED;
+  const long cache_rows = long(num_blocks) * Hkv * 16;
+  if (cache_rows > 0x7fffffffL || long(max_blocks_per_seq) * 16 > 0x7fffffffL) return FA_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  CUtensorMap mq, mk, mv, mo;
+  if (!make_map_bf16(&mq, q, d, Nq_max, R * Hq, 128) || !make_map_bf16(&mo, o, d, Nq_max, R * Hq, 32) ||
+      !make_map_cache(&mk, k_cache, cache_rows, d) || !make_map_cache(&mv, v_cache, cache_rows, d))
+    return FA_ERR_CUDA;
+  FwdBf16Params prm{static_cast<__nv_bfloat16*>(o), lse, R * Hq, Hq, Hkv, Nq_max, 0,
+                    scale * 1.4426950408889634f, g_wait_ns, block_table, ctx_lens, q_lens, max_blocks_per_seq,
+                    num_blocks};
+  constexpr int BN64 = FA_FWD_D64_BN;
+  if (d == 64)
+    return causal ? launch_fwd_bf16<64, BN64, true, true>(mq, mk, mv, mo, prm, Nq_max, st)
+                  : launch_fwd_bf16<64, BN64, false, true>(mq, mk, mv, mo, prm, Nq_max, st);
+  return causal ? launch_fwd_bf16<128, 128, true, true>(mq, mk, mv, mo, prm, Nq_max, st)
+                : launch_fwd_bf16<128, 128, false, true>(mq, mk, mv, mo, prm, Nq_max, st);
 }
 
 size_t fa_bwd_workspace_size(int B, int Hq, int Nq, int d) {

@@ -82,6 +82,11 @@ struct FwdBf16Params {
   int BH, Hq, Hkv, Nq, Nkv;
   float scale_log2;  // scale * log2(e)
   uint64_t wait_ns;
+  // paged mode (prefill over a paged KV cache): per-request lengths and the block table
+  const int* bt;
+  const int* ctx;   // cached tokens of request b (the keys)
+  const int* qlen;  // query rows of request b (the last qlen positions of its sequence)
+  int max_blocks, num_blocks;
 };
 
 struct FwdBars {
@@ -97,7 +102,7 @@ struct FwdBars {
   int abort_flag;
 };
 
-template <int D, int BN, bool CAUSAL>
+template <int D, int BN, bool CAUSAL, bool PAGED>
 __global__ void __launch_bounds__(FwdCfg<D, BN>::THREADS, FwdCfg<D, BN>::CTAS_PER_SM)
     fa_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -111,18 +116,53 @@ __global__ void __launch_bounds__(FwdCfg<D, BN>::THREADS, FwdCfg<D, BN>::CTAS_PE
   const int warp = warp_id(), lane = lane_id();
   const int n_qp = (p.Nq + 2 * C::BM - 1) / (2 * C::BM);
   const int n_items = n_qp * p.BH;
-  const int off = p.Nkv - p.Nq;  // bottom-right causal alignment
   // item -> (query-tile pair, batch*head).  Non-causal items are head-major, so the CTAs
   // running at the same time share one or two heads' K/V in L2 (at N = 8192 this cut
   // DRAM traffic per launch from 4.2 GB to the 0.64 GB of the algorithm); causal items are
   // longest-first over all heads (last query tiles first), which balances their very
   // unequal lengths better than any head grouping measured.
-  auto item_qt = [&](int it) { return CAUSAL ? n_qp - 1 - it / p.BH : it % n_qp; };
-  auto item_bh = [&](int it) { return CAUSAL ? it % p.BH : it / n_qp; };
-  auto item_ntiles = [&](int qt) {
-    int kv_end = p.Nkv;
-    if (CAUSAL) kv_end = min(p.Nkv, min(qt * 2 * C::BM + 2 * C::BM, p.Nq) + off);
-    return (kv_end + C::BN - 1) / C::BN;
+  // keys (L) and query rows (ql) of a sequence; paged mode reads them per request and
+  // gives out-of-range lengths no work (flagging them in the status word)
+  auto seq_len = [&](int bh, int& L, int& ql) {
+    if constexpr (PAGED) {
+      const int r = bh / p.Hq;
+      L = __ldg(p.ctx + r);
+      ql = __ldg(p.qlen + r);
+      if (L < 1 || L > p.max_blocks * 16 || ql < 1 || ql > L || ql > p.Nq) {
+        if (threadIdx.x == 0 && bh % p.Hq == 0) set_status(FA_ERR_INVALID_ARG, 60);
+        L = 0;
+        ql = 0;
+      }
+    } else {
+      L = p.Nkv;
+      ql = p.Nq;
+    }
+  };
+  // item -> (query-tile pair qt, batch*head bh, its sequence's L and ql, key tiles n; n = 0:
+  // nothing to do).  Non-causal items are head-major, so the CTAs running at the same time
+  // share one or two heads' K/V in L2 (at N = 8192 this cut DRAM traffic per launch from
+  // 4.2 GB to the 0.64 GB of the algorithm); causal items are longest-first over all heads
+  // (last query tiles first), which balances their very unequal lengths better than any
+  // head grouping measured.  In paged mode the causal order counts tile pairs from each
+  // request's own last one, so the long items of every request come first.
+  struct Item {
+    int qt, bh, L, ql, n;
+  };
+  auto item_of = [&](int it) {
+    Item x;
+    x.bh = CAUSAL ? it % p.BH : it / n_qp;
+    seq_len(x.bh, x.L, x.ql);
+    if (CAUSAL && PAGED)
+      x.qt = (x.ql + 2 * C::BM - 1) / (2 * C::BM) - 1 - it / p.BH;
+    else
+      x.qt = CAUSAL ? n_qp - 1 - it / p.BH : it % n_qp;
+    x.n = 0;
+    if (x.qt >= 0 && x.qt * 2 * C::BM < x.ql) {
+      int kv_end = x.L;
+      if (CAUSAL) kv_end = min(x.L, min(x.qt * 2 * C::BM + 2 * C::BM, x.ql) + (x.L - x.ql));
+      x.n = (kv_end + C::BN - 1) / C::BN;
+    }
+    return x;
   };
 
   if (threadIdx.x == 0) {
@@ -156,7 +196,7 @@ __global__ void __launch_bounds__(FwdCfg<D, BN>::THREADS, FwdCfg<D, BN>::CTAS_PE
   const uint32_t sK = smem_u32(smem + C::OFF_K);
   const uint32_t sV = smem_u32(smem + C::OFF_V);
 
-  if (warp == 0) {
+  if (warp == 0 && !PAGED) {
     // ---------------------------------------------------------------- TMA producer
     if (lane == 0) {
       prefetch_tmap(&tmQ);
@@ -165,19 +205,19 @@ __global__ void __launch_bounds__(FwdCfg<D, BN>::THREADS, FwdCfg<D, BN>::CTAS_PE
       int kv = 0;  // K/V tiles issued so far (ring position)
       int local = 0;
       bool ok = true;
-      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++local) {
-        const int qt = item_qt(it), bh = item_bh(it);
-        const int b = bh / p.Hq, h = bh % p.Hq;
-        const int zkv = b * p.Hkv + h / (p.Hq / p.Hkv);
-        const int n = item_ntiles(qt);
+      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+        const Item x = item_of(it);
+        if (x.n == 0) continue;
+        const int zkv = (x.bh / p.Hq) * p.Hkv + (x.bh % p.Hq) / (p.Hq / p.Hkv);
         const int qb = local % C::QBUF, quse = local / C::QBUF;
+        ++local;
         if (quse > 0 && !(ok = mbar_wait(&bars->q_empty[qb], (quse - 1) & 1, p.wait_ns, abort_flag, 11))) break;
         mbar_arrive_expect_tx(&bars->q_full[qb], 2 * C::Q_TILE);
         for (int t = 0; t < 2; ++t)
           for (int kb = 0; kb < C::KB; ++kb)
             tma_load_3d(smem + C::OFF_Q + (qb * 2 + t) * C::Q_TILE + kb * C::BM * 128, &tmQ, &bars->q_full[qb],
-                        kb * 64, qt * 2 * C::BM + t * C::BM, bh);
-        for (int j = 0; j < n; ++j, ++kv) {
+                        kb * 64, x.qt * 2 * C::BM + t * C::BM, x.bh);
+        for (int j = 0; j < x.n; ++j, ++kv) {
           const int st = kv % C::NSTAGE, round = kv / C::NSTAGE;
           if (round > 0 && !(ok = mbar_wait(&bars->kv_empty[st], (round - 1) & 1, p.wait_ns, abort_flag, 10)))
             break;
@@ -190,6 +230,76 @@ __global__ void __launch_bounds__(FwdCfg<D, BN>::THREADS, FwdCfg<D, BN>::CTAS_PE
             tma_load_3d(smem + C::OFF_V + st * C::KV_TILE + kb * C::BN * 128, &tmV, &bars->v_full[st], kb * 64,
                         j * C::BN, zkv);
         }
+      }
+    }
+  } else if (warp == 0) {
+    // ------------------------------------------------- TMA producer, paged K/V (whole warp)
+    // A tile's BN keys are NB = BN/16 cache blocks.  Lane i < NB owns block i of the tile:
+    // it reads the block-table entry one tile ahead and issues that block's 16-row boxes
+    // (one per 64-column block of K and of V) at the physical rows the entry gives.
+    // Blocks past the sequence are not loaded: their V rows are zeroed (their P is 0, and
+    // 0 * NaN would not be), their K rows keep stale data (those scores are masked).
+    constexpr int NB = C::BN / 16;
+    if (lane == 0) {
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+    }
+    int kv = 0, local = 0;
+    bool ok = true;
+    for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+      const Item x = item_of(it);
+      if (x.n == 0) continue;
+      const int b = x.bh / p.Hq;
+      const int hk = (x.bh % p.Hq) / (p.Hq / p.Hkv);
+      const int* bt = p.bt + size_t(b) * p.max_blocks;
+      const int nblk = (x.L + 15) / 16;
+      int ph = (lane < NB && lane < nblk) ? __ldg(bt + lane) : 0;  // entry for tile 0
+      const int qb = local % C::QBUF, quse = local / C::QBUF;
+      ++local;
+      if (quse > 0 && !(ok = warp_wait(&bars->q_empty[qb], (quse - 1) & 1, p.wait_ns, abort_flag, 11))) break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&bars->q_full[qb], 2 * C::Q_TILE);
+        for (int t = 0; t < 2; ++t)
+          for (int kb = 0; kb < C::KB; ++kb)
+            tma_load_3d(smem + C::OFF_Q + (qb * 2 + t) * C::Q_TILE + kb * C::BM * 128, &tmQ, &bars->q_full[qb],
+                        kb * 64, x.qt * 2 * C::BM + t * C::BM, x.bh);
+      }
+      for (int j = 0; j < x.n; ++j, ++kv) {
+        const int st = kv % C::NSTAGE, round = kv / C::NSTAGE;
+        const int lb = j * NB + lane;
+        const int ph_next = (lane < NB && lb + NB < nblk) ? __ldg(bt + lb + NB) : 0;
+        if (round > 0 && !(ok = warp_wait(&bars->kv_empty[st], (round - 1) & 1, p.wait_ns, abort_flag, 10))) break;
+        uint8_t* sk = smem + C::OFF_K + st * C::KV_TILE;
+        uint8_t* sv = smem + C::OFF_V + st * C::KV_TILE;
+        const int nload = min(NB, nblk - j * NB);  // >= 1: every tile starts inside the sequence
+        if (nload < NB) {
+          const int z0 = nload * 16 * 8, z1 = C::BN * 8;  // 16-byte units of one 64-column block
+          for (int kb = 0; kb < C::KB; ++kb)
+            for (int i = z0 + lane; i < z1; i += 32)
+              *reinterpret_cast<uint4*>(sv + kb * C::BN * 128 + i * 16) = make_uint4(0, 0, 0, 0);
+          fence_proxy_async_smem();
+        }
+        __syncwarp();
+        if (lane == 0) {
+          const uint32_t bytes = uint32_t(nload) * 16 * 128 * C::KB;
+          mbar_arrive_expect_tx(&bars->k_full[st], bytes);
+          mbar_arrive_expect_tx(&bars->v_full[st], bytes);
+        }
+        __syncwarp();
+        if (lane < nload) {
+          int pb = ph;
+          if (pb < 0 || pb >= p.num_blocks) {  // a bad table entry: flagged, block 0 read instead
+            set_status(FA_ERR_INVALID_ARG, 61);
+            pb = 0;
+          }
+          const int crow = (pb * p.Hkv + hk) * 16;
+          for (int kb = 0; kb < C::KB; ++kb) {
+            tma_load_2d(smem_u32(sk + kb * C::BN * 128 + lane * 16 * 128), &tmK, &bars->k_full[st], kb * 64, crow);
+            tma_load_2d(smem_u32(sv + kb * C::BN * 128 + lane * 16 * 128), &tmV, &bars->v_full[st], kb * 64, crow);
+          }
+        }
+        ph = ph_next;
       }
     }
   } else if (warp == 1) {
@@ -219,10 +329,13 @@ __global__ void __launch_bounds__(FwdCfg<D, BN>::THREADS, FwdCfg<D, BN>::CTAS_PE
       int g = 0;   // query-tile steps so far (s_full / p_full phase)
       int local = 0;
       bool ok = true;
-      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++local) {
-        const int n = item_ntiles(item_qt(it));
-        const int qb = local % C::QBUF;
-        ok = mbar_wait(&bars->q_full[qb], (local / C::QBUF) & 1, p.wait_ns, abort_flag, 20) &&
+      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+        const Item x = item_of(it);
+        const int n = x.n, L = x.L;
+        if (n == 0) continue;
+        const int qb = local % C::QBUF, quse = local / C::QBUF;
+        ++local;
+        ok = mbar_wait(&bars->q_full[qb], quse & 1, p.wait_ns, abort_flag, 20) &&
              mbar_wait(&bars->k_full[kv % C::NSTAGE], (kv / C::NSTAGE) & 1, p.wait_ns, abort_flag, 21);
         if (!ok) break;
         tc_fence_after();
@@ -234,8 +347,22 @@ __global__ void __launch_bounds__(FwdCfg<D, BN>::THREADS, FwdCfg<D, BN>::CTAS_PE
           const int st = kv % C::NSTAGE;
           const int st2 = (kv + 1) % C::NSTAGE;
           const bool more = j + 1 < n;
-          ok = mbar_wait(&bars->v_full[st], (kv / C::NSTAGE) & 1, p.wait_ns, abort_flag, 22) &&
-               mbar_wait(&bars->p_full[0], g & 1, p.wait_ns, abort_flag, 23);
+          ok = mbar_wait(&bars->v_full[st], (kv / C::NSTAGE) & 1, p.wait_ns, abort_flag, 22);
+          if (!ok) break;
+          if constexpr (PAGED) {
+            // the sequence's last cache block is partly filled: zero the V rows of its
+            // unused slots (loaded with the block; their P is 0, and 0 * NaN would not be)
+            const int last = (L - 1) / 16;
+            if ((L & 15) != 0 && last / (C::BN / 16) == j) {
+              uint8_t* sv = smem + C::OFF_V + st * C::KV_TILE;
+              const int r0 = L - j * C::BN, r1 = (last + 1) * 16 - j * C::BN;
+              for (int kb = 0; kb < C::KB; ++kb)
+                for (int i = r0 * 8; i < r1 * 8; ++i)
+                  *reinterpret_cast<uint4*>(sv + kb * C::BN * 128 + i * 16) = make_uint4(0, 0, 0, 0);
+              fence_proxy_async_smem();
+            }
+          }
+          ok = mbar_wait(&bars->p_full[0], g & 1, p.wait_ns, abort_flag, 23);
           if (!ok) break;
           tc_fence_after();
           issue_PV(0, st, j);
@@ -274,15 +401,17 @@ __global__ void __launch_bounds__(FwdCfg<D, BN>::THREADS, FwdCfg<D, BN>::CTAS_PE
     const float sl2 = p.scale_log2;
     int g = 0, local = 0;
     bool ok = true;
-    for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++local) {
-      const int qt = item_qt(it), bh = item_bh(it);
-      const int n = item_ntiles(qt);
+    for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+      const Item x = item_of(it);
+      const int qt = x.qt, bh = x.bh, L = x.L, ql = x.ql, n = x.n;
+      if (n == 0) continue;
+      const int item_local = local++;
       const int row = qt * 2 * C::BM + t * C::BM + r;
-      const int row_limit = CAUSAL ? min(p.Nkv, row + off + 1) : p.Nkv;
+      const int row_limit = CAUSAL ? min(L, row + (L - ql) + 1) : L;
       float m = -INFINITY, l = 0.f;
-      // a warp whose rows are all padding (past Nq) skips the arithmetic: its P rows
-      // only feed output rows that are never stored
-      const bool idle = __all_sync(0xffffffffu, row >= p.Nq);
+      // a warp whose rows are all padding (past the query rows) skips the arithmetic: its
+      // P rows only feed output rows that are never part of the result
+      const bool idle = __all_sync(0xffffffffu, row >= ql);
       for (int j = 0; j < n; ++j, ++g) {
         ok = warp_wait(&bars->s_full[t], g & 1, p.wait_ns, abort_flag, 30 + t);
         if (!ok) break;
@@ -384,7 +513,7 @@ __global__ void __launch_bounds__(FwdCfg<D, BN>::THREADS, FwdCfg<D, BN>::CTAS_PE
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->p_full[t]);
       }
-      if (ok) ok = warp_wait(&bars->o_final[t], local & 1, p.wait_ns, abort_flag, 40 + t);
+      if (ok) ok = warp_wait(&bars->o_final[t], item_local & 1, p.wait_ns, abort_flag, 40 + t);
       if (!ok) break;
       if (idle) continue;
       tc_fence_after();
@@ -422,7 +551,7 @@ __global__ void __launch_bounds__(FwdCfg<D, BN>::THREADS, FwdCfg<D, BN>::CTAS_PE
           bulk_commit();
         }
       }
-      if (row < p.Nq) p.lse[size_t(bh) * p.Nq + row] = (m + __log2f(l)) * 0.69314718055994531f;
+      if (row < ql) p.lse[size_t(bh) * p.Nq + row] = (m + __log2f(l)) * 0.69314718055994531f;
     }
     if (lane == 0) bulk_wait_all();
   }

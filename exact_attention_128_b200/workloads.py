@@ -94,6 +94,40 @@ def prefill_sweep():
     return out
 
 
+def paged_pool(ctx, block_size: int, max_blocks_per_seq: int, Hkv: int, d: int, g: torch.Generator, s: int,
+               poison_unused: bool):
+    """Lay R sequences of ``ctx`` tokens out in a paged K/V pool.
+
+    The pool holds exactly sum_r ceil(ctx_r / block_size) blocks; a random permutation
+    (drawn from ``g``) assigns a physical id to each (request, logical block) pair in
+    order.  Table entries past a request's last block are -1.  Caches are
+    [blocks, Hkv, block_size, d] bf16 drawn with seeds s + 2 (K) and s + 3 (V).  With
+    ``poison_unused`` the unused slots of each request's last block hold NaN.
+    Returns (table, k_cache, v_cache, num_blocks).
+    """
+    R = len(ctx)
+    nblk = [(int(c) + block_size - 1) // block_size for c in ctx]
+    total = sum(nblk)
+    if max(nblk) > max_blocks_per_seq:
+        raise ValueError("context longer than the block table allows")
+    perm = torch.randperm(total, generator=g)
+    table = torch.full((R, max_blocks_per_seq), -1, dtype=torch.int32)
+    pos = 0
+    for r in range(R):
+        table[r, : nblk[r]] = perm[pos : pos + nblk[r]].to(torch.int32)
+        pos += nblk[r]
+    kc = randn((total, Hkv, block_size, d), s + 2, torch.bfloat16)
+    vc = randn((total, Hkv, block_size, d), s + 3, torch.bfloat16)
+    if poison_unused:
+        for r in range(R):
+            used = int(ctx[r]) - (nblk[r] - 1) * block_size
+            if used < block_size:
+                pb = int(table[r, nblk[r] - 1])
+                kc[pb, :, used:, :] = float("nan")
+                vc[pb, :, used:, :] = float("nan")
+    return table, kc, vc, total
+
+
 @dataclass
 class PagedCase:
     """One paged-KV decode step: R requests with one new query token each."""
@@ -129,27 +163,9 @@ class PagedCase:
             ctx = torch.tensor(self.ctx_lens_override, dtype=torch.int32)
         else:
             ctx = torch.randint(self.ctx_min, self.ctx_max + 1, (self.R,), generator=g, dtype=torch.int64).to(torch.int32)
-        nblk = [(int(c) + self.block_size - 1) // self.block_size for c in ctx]
-        total = sum(nblk)
-        if max(nblk) > self.max_blocks_per_seq:
-            raise ValueError("context longer than the block table allows")
-        perm = torch.randperm(total, generator=g)
-        table = torch.full((self.R, self.max_blocks_per_seq), -1, dtype=torch.int32)
-        pos = 0
-        for r in range(self.R):
-            table[r, : nblk[r]] = perm[pos : pos + nblk[r]].to(torch.int32)
-            pos += nblk[r]
-        s = self.seed * 1000
-        q = randn((self.R, self.Hq, self.d), s + 1, torch.bfloat16)
-        kc = randn((total, self.Hkv, self.block_size, self.d), s + 2, torch.bfloat16)
-        vc = randn((total, self.Hkv, self.block_size, self.d), s + 3, torch.bfloat16)
-        if poison_unused:
-            for r in range(self.R):
-                used = int(ctx[r]) - (nblk[r] - 1) * self.block_size
-                if used < self.block_size:
-                    pb = int(table[r, nblk[r] - 1])
-                    kc[pb, :, used:, :] = float("nan")
-                    vc[pb, :, used:, :] = float("nan")
+        table, kc, vc, total = paged_pool(ctx, self.block_size, self.max_blocks_per_seq, self.Hkv, self.d, g,
+                                          self.seed * 1000, poison_unused)
+        q = randn((self.R, self.Hq, self.d), self.seed * 1000 + 1, torch.bfloat16)
         return {"q": q, "k_cache": kc, "v_cache": vc, "block_table": table, "ctx_lens": ctx, "num_blocks": total}
 
     @staticmethod
@@ -160,3 +176,87 @@ class PagedCase:
 
 # 1.5B-class decoder decode step: 64 requests, Hq = 12, Hkv = 2, d = 128, 16-token blocks.
 PAGED_DECODE = PagedCase("paged_decode_r64_hq12_hkv2_d128_bs16", 64, 12, 2, 128, 16, 512, 8192, 512, 5)
+
+
+@dataclass
+class PagedPrefillCase:
+    """A batch of variable-length prefills over a paged KV cache.
+
+    Request r has ctx_r cached tokens and q_r query rows, the last q_r positions of its
+    sequence: q_r = ctx_r for a whole prompt (``q_frac`` = 1), else a seeded chunk
+    length q_r ~ U{1..max(1, round(q_frac * ctx_r))}.  q is [R, Hq, Nq_max, d] with
+    Nq_max = max_r q_r; rows past q_r are padding.
+    """
+
+    name: str
+    R: int
+    Hq: int
+    Hkv: int
+    d: int
+    block_size: int
+    ctx_min: int
+    ctx_max: int
+    max_blocks_per_seq: int
+    causal: bool
+    seed: int
+    q_frac: float = 1.0
+    ctx_lens_override: tuple | None = None
+    q_lens_override: tuple | None = None
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    def lengths(self):
+        g = torch.Generator().manual_seed(self.seed * 1000)
+        if self.ctx_lens_override is not None:
+            ctx = torch.tensor(self.ctx_lens_override, dtype=torch.int32)
+        else:
+            ctx = torch.randint(self.ctx_min, self.ctx_max + 1, (self.R,), generator=g, dtype=torch.int64).to(torch.int32)
+        if self.q_lens_override is not None:
+            ql = torch.tensor(self.q_lens_override, dtype=torch.int32)
+        elif self.q_frac >= 1.0:
+            ql = ctx.clone()
+        else:
+            hi = [max(1, round(self.q_frac * int(c))) for c in ctx]
+            ql = torch.tensor([int(torch.randint(1, h + 1, (1,), generator=g)) for h in hi], dtype=torch.int32)
+        return ctx, ql, g
+
+    def make(self, poison: bool = False):
+        """Return dict with q, k_cache, v_cache, block_table, ctx_lens, q_lens, num_blocks (CPU).
+
+        With ``poison`` the unused cache slots of each last block and the padding query
+        rows hold NaN (a correct kernel never reads them into the result)."""
+        ctx, ql, g = self.lengths()
+        s = self.seed * 1000
+        table, kc, vc, total = paged_pool(ctx, self.block_size, self.max_blocks_per_seq, self.Hkv, self.d, g, s,
+                                          poison)
+        nq_max = int(ql.max())
+        q = randn((self.R, self.Hq, nq_max, self.d), s + 1, torch.bfloat16)
+        if poison:
+            for r in range(self.R):
+                q[r, :, int(ql[r]):, :] = float("nan")
+        return {"q": q, "k_cache": kc, "v_cache": vc, "block_table": table, "ctx_lens": ctx, "q_lens": ql,
+                "num_blocks": total}
+
+    def allowed_pairs(self) -> int:
+        """(query, key) pairs the prefill computes, summed over requests (per head)."""
+        ctx, ql, _ = self.lengths()
+        tot = 0
+        for c, n in zip(ctx.tolist(), ql.tolist()):
+            tot += n * (2 * c - n + 1) // 2 if self.causal else n * c
+        return tot
+
+    def fwd_flops(self) -> float:
+        return 4.0 * self.d * self.Hq * self.allowed_pairs()
+
+    def io_bytes(self) -> int:
+        """Algorithmic bytes: every cached K/V row once per KV head, q and o rows once (bf16)."""
+        ctx, ql, _ = self.lengths()
+        return int(ctx.sum()) * self.Hkv * self.d * 2 * 2 + int(ql.sum()) * self.Hq * self.d * 2 * 2
+
+
+# Paged counterpart of the causal GQA prefill: 8 whole prompts of U{2048..8192} tokens,
+# Hq = 32, Hkv = 8, d = 128, 16-token blocks.
+PAGED_PREFILL = PagedPrefillCase("paged_prefill_r8_hq32_hkv8_d128_bs16_causal", 8, 32, 8, 128, 16, 2048, 8192, 512,
+                                 True, 6)

@@ -132,6 +132,36 @@ fa_status fa_paged_decode(const void* q, const void* k_cache, const void* v_cach
                           void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * fa_paged_prefill — forward pass of a batch of variable-length sequences whose keys and
+ * values sit in a paged KV cache ("Atención tipo FlashAttention y atención paginada": a
+ * block table links logical positions to fixed-size physical blocks; the same page's
+ * tiled online-softmax forward is run over the blocks the table names).
+ *   Request r has ctx_lens[r] cached tokens (its keys and values, already written to the
+ *   cache, e.g. by fa_paged_kv_append) and q_lens[r] query rows, which are the LAST
+ *   q_lens[r] positions of its sequence (1 <= q_lens[r] <= ctx_lens[r]; equal for a
+ *   fresh prompt, smaller for a chunk of a prompt whose earlier part is cached).
+ *   q [R,Hq,Nq_max,d] bf16: query row i of request r at q[r,:,i,:], i < q_lens[r];
+ *     q_lens[r] <= Nq_max.  Rows i >= q_lens[r] are not read into any result.
+ *   k_cache, v_cache [num_blocks, Hkv, block_size, d] bf16; block_table [R,
+ *     max_blocks_per_seq] int32 (entries at or past ceil(ctx_lens[r] / block_size) are
+ *     never read); ctx_lens, q_lens [R] int32 (device).
+ *   causal: 1 = query row i sees keys j <= i + ctx_lens[r] - q_lens[r] (its own position
+ *     and every earlier one); 0 = it sees all ctx_lens[r] keys.
+ *   o [R,Hq,Nq_max,d] bf16 and lse [R,Hq,Nq_max] fp32 (natural log): rows i >= q_lens[r]
+ *     are left undefined (o) or untouched (lse).
+ *   d == 64 or 128, block_size == 16, GQA as in fa_fwd.
+ *   A length or block id out of range is not dereferenced: the kernel skips that request
+ *   (or reads block 0 for the bad entry) and sets the device status word
+ *   (FA_ERR_INVALID_ARG), so that request's result is undefined.
+ * Errors: FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA.
+ */
+fa_status fa_paged_prefill(const void* q, const void* k_cache, const void* v_cache,
+                           const int* block_table, const int* ctx_lens, const int* q_lens,
+                           void* o, float* lse, int R, int Hq, int Hkv, int Nq_max, int d,
+                           int block_size, int max_blocks_per_seq, int num_blocks, float scale,
+                           int causal, fa_dtype dtype, void* stream);
+
+/*
  * fa_paged_kv_append — writes one new token per request into a paged KV cache ("Atención
  * tipo FlashAttention y atención paginada": the cache grows one token at a time and the
  * block table links logical positions to fixed-size physical blocks).

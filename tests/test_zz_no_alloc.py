@@ -58,8 +58,8 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls():
 def test_noalloc_rejects_requests_beyond_its_scratch():
     L = fa.lib()
     fake = ctypes.c_void_p(1 << 20)  # rejected on the host before any use
-    need = L.fa_paged_decode_workspace_size(64, 12, 128, 2048, 16)
+    need = L.fa_paged_decode_workspace_size(64, 12, 128, 8192, 16)
     assert need > 8 * 1024 * 1024
-    st = L.fa_paged_decode_noalloc(fake, fake, fake, fake, fake, fake, None, 64, 12, 2, 128, 16, 2048, 40000,
+    st = L.fa_paged_decode_noalloc(fake, fake, fake, fake, fake, fake, None, 64, 12, 2, 128, 16, 8192, 40000,
                                    ctypes.c_float(0.088), fa.FA_DTYPE_BF16, None)
     assert st == fa.FA_ERR_WORKSPACE
