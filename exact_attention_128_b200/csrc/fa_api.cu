@@ -10,10 +10,12 @@
 #include "fwd_bf16.cuh"
 #include "fwd_f32.cuh"
 #include "bwd_bf16.cuh"
+#include "bwd_f32.cuh"
 
 #ifndef FA_FWD_D64_BN
 #define FA_FWD_D64_BN 64
 #endif
+
 
 namespace {
 
@@ -41,17 +43,20 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 3-D bf16 map over [z][y][x] = [planes][rows][d] with a (64, box_rows, 1) box and the
-// 128-byte swizzle; rows past `rows` read as zeros.
-bool make_map_bf16(CUtensorMap* m, const void* base, int d, int rows, int planes, int box_rows) {
+// 3-D bf16 map over [z][y][x] = [planes][rows][d] with a (box_cols, box_rows, 1) box and
+// the swizzle of its row width (64 columns: 128-byte, 32 columns: 64-byte); rows past
+// `rows` read as zeros.
+bool make_map_bf16(CUtensorMap* m, const void* base, int d, int rows, int planes, int box_rows,
+                   int box_cols = 64) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(rows), cuuint64_t(planes)};
   cuuint64_t strides[2] = {cuuint64_t(d) * 2, cuuint64_t(d) * 2 * cuuint64_t(rows)};
-  cuuint32_t box[3] = {64, cuuint32_t(box_rows), 1};
+  cuuint32_t box[3] = {cuuint32_t(box_cols), cuuint32_t(box_rows), 1};
   cuuint32_t estr[3] = {1, 1, 1};
+  const CUtensorMapSwizzle sw = box_cols == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -263,13 +268,17 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
     return launched();
   }
   if (dtype != FA_DTYPE_BF16) return FA_ERR_UNSUPPORTED;
-  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 96 && d != 128) return FA_ERR_UNSUPPORTED;
 
   constexpr int BN64 = FA_FWD_D64_BN;  // key-tile width of the d = 64 kernel
   const int bn = d == 64 ? BN64 : 128;
+  const int stg_cols = d == 64 ? FwdCfg<64, BN64>::STG_COLS : FwdCfg<128, 128>::STG_COLS;
+  // d = 96 runs the d = 128 kernel: the maps' rows are 96 wide, so TMA loads fill columns
+  // 96..127 with zeros (adding nothing to Q K^T, giving zero columns of O) and the O stores
+  // drop them
   CUtensorMap mq, mk, mv, mo;
   if (!make_map_bf16(&mq, q, d, Nq, B * Hq, 128) || !make_map_bf16(&mk, k, d, Nkv, B * Hkv, bn) ||
-      !make_map_bf16(&mv, v, d, Nkv, B * Hkv, bn) || !make_map_bf16(&mo, o, d, Nq, B * Hq, 32))
+      !make_map_bf16(&mv, v, d, Nkv, B * Hkv, bn) || !make_map_bf16(&mo, o, d, Nq, B * Hq, 32, stg_cols))
     return FA_ERR_CUDA;
   FwdBf16Params prm{static_cast<__nv_bfloat16*>(o), lse, B * Hq, Hq, Hkv, Nq, Nkv,
                     scale * 1.4426950408889634f, g_wait_ns, nullptr, nullptr, nullptr, 0, 0};
@@ -294,19 +303,20 @@ fa_status fa_paged_prefill(const void* q, const void* k_cache, const void* v_cac
   if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(o, 16) || !aligned(lse, 4) ||
       !aligned(block_table, 4) || !aligned(ctx_lens, 4) || !aligned(q_lens, 4))
     return FA_ERR_INVALID_ARG;
-  if (dtype != FA_DTYPE_BF16 || (d != 64 && d != 128) || block_size != 16) return FA_ERR_UNSUPPORTED;
+  if (dtype != FA_DTYPE_BF16 || (d != 64 && d != 96 && d != 128) || block_size != 16) return FA_ERR_UNSUPPORTED;
   if (long(R) * Hq > 65535) return FA_ERR_UNSUPPORTED;
   const long cache_rows = long(num_blocks) * Hkv * 16;
   if (cache_rows > 0x7fffffffL || long(max_blocks_per_seq) * 16 > 0x7fffffffL) return FA_ERR_UNSUPPORTED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   CUtensorMap mq, mk, mv, mo;
-  if (!make_map_bf16(&mq, q, d, Nq_max, R * Hq, 128) || !make_map_bf16(&mo, o, d, Nq_max, R * Hq, 32) ||
+  constexpr int BN64 = FA_FWD_D64_BN;
+  const int stg_cols = d == 64 ? FwdCfg<64, BN64>::STG_COLS : FwdCfg<128, 128>::STG_COLS;
+  if (!make_map_bf16(&mq, q, d, Nq_max, R * Hq, 128) || !make_map_bf16(&mo, o, d, Nq_max, R * Hq, 32, stg_cols) ||
       !make_map_cache(&mk, k_cache, cache_rows, d) || !make_map_cache(&mv, v_cache, cache_rows, d))
     return FA_ERR_CUDA;
   FwdBf16Params prm{static_cast<__nv_bfloat16*>(o), lse, R * Hq, Hq, Hkv, Nq_max, 0,
                     scale * 1.4426950408889634f, g_wait_ns, block_table, ctx_lens, q_lens, max_blocks_per_seq,
                     num_blocks};
-  constexpr int BN64 = FA_FWD_D64_BN;
   if (d == 64)
     return causal ? launch_fwd_bf16<64, BN64, true, true>(mq, mk, mv, mo, prm, Nq_max, st)
                   : launch_fwd_bf16<64, BN64, false, true>(mq, mk, mv, mo, prm, Nq_max, st);
@@ -334,6 +344,23 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   for (const void* ptr : ptrs)
     if (!aligned(ptr, 16)) return FA_ERR_INVALID_ARG;
   if (!aligned(lse, 4)) return FA_ERR_INVALID_ARG;
+  if (dtype == FA_DTYPE_F32) {
+    // fp32 inputs: CUDA-core kernels (bwd_f32.cuh), fp32 gradients, d = 64
+    if (d != b32::D || grad_dtype != FA_DTYPE_F32) return FA_ERR_UNSUPPORTED;
+    if (long(B) * Hq > 65535 || long(B) * Hkv > 65535) return FA_ERR_UNSUPPORTED;
+    const long rows = long(B) * Hq * Nq;
+    if (!workspace || workspace_bytes < fa_bwd_workspace_size(B, Hq, Nq, d) || !aligned(workspace, 256))
+      return FA_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    BwdF32Params prm{static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
+                     static_cast<const float*>(o), lse, static_cast<const float*>(dO), static_cast<float*>(dq),
+                     static_cast<float*>(dk), static_cast<float*>(dv), static_cast<float*>(workspace), Hq, Hkv, Nq,
+                     Nkv, scale, causal};
+    fa_bwd_f32_pre_kernel<<<unsigned((rows + 7) / 8), 256, 0, st>>>(prm.o, prm.dO, prm.Dvec, rows);
+    fa_bwd_f32_dkdv_kernel<<<dim3((Nkv + b32::BK - 1) / b32::BK, B * Hkv), b32::THREADS, 0, st>>>(prm);
+    fa_bwd_f32_dq_kernel<<<dim3((Nq + b32::BQ - 1) / b32::BQ, B * Hq), b32::THREADS, 0, st>>>(prm);
+    return launched();
+  }
   if (dtype != FA_DTYPE_BF16) return FA_ERR_UNSUPPORTED;
   if (grad_dtype != FA_DTYPE_F32 && grad_dtype != FA_DTYPE_BF16) return FA_ERR_UNSUPPORTED;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;

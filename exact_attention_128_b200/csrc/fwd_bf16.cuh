@@ -53,6 +53,17 @@ namespace fa {
 //            shared memory, so two CTAs share an SM and four query tiles are in flight;
 //            at d = 64 the softmax, not the tensor core, sets the pace, and the second
 //            CTA hides its latency.
+// d = 64 kernel: K/V ring depth and the output columns a softmax warp stages per TMA store
+// (64: 4 KB per warp, 128-byte swizzle; 32: 2 KB per warp, 64-byte swizzle, two stores).
+// Measured on B200: 32-column staging 3-5 % faster (ViT-B/16 layer 34.8 -> 33.1 us, N = 4096
+// causal 441 -> 426 us); 3 or 4 stages no faster than 2.
+#ifndef FA_FWD_D64_NSTAGE
+#define FA_FWD_D64_NSTAGE 2
+#endif
+#ifndef FA_FWD_D64_STG_COLS
+#define FA_FWD_D64_STG_COLS 32
+#endif
+
 template <int D, int BN_>
 struct FwdCfg {
   static constexpr int BM = 128;   // rows per query tile (two tiles per item)
@@ -61,16 +72,25 @@ struct FwdCfg {
   static constexpr int Q_TILE = BM * D * 2;
   static constexpr int KV_TILE = BN * D * 2;
   static constexpr int QBUF = (D == 128 || BN == 64) ? 1 : 2;
-  static constexpr int NSTAGE = (BN == 64) ? 2 : (D == 128 ? 2 : 4);
+  static constexpr int NSTAGE = (BN == 64) ? FA_FWD_D64_NSTAGE : (D == 128 ? 2 : 4);
+  static constexpr int STG_COLS = (BN == 64) ? FA_FWD_D64_STG_COLS : 64;
+  static constexpr int STG_WARP = 32 * STG_COLS * 2;  // staging bytes per softmax warp
   static constexpr int OFF_Q = 0;  // + qb * 2 * Q_TILE + t * Q_TILE
   static constexpr int OFF_K = QBUF * 2 * Q_TILE;
   static constexpr int OFF_V = OFF_K + NSTAGE * KV_TILE;
-  static constexpr int OFF_STG = OFF_V + NSTAGE * KV_TILE;  // epilogue staging: 4 KB per softmax warp
-  static constexpr int OFF_BAR = OFF_STG + 8 * 4096;
-  static constexpr int SMEM = OFF_BAR + 256 + 1024;  // + barriers + alignment slack
+  static constexpr int OFF_STG = OFF_V + NSTAGE * KV_TILE;  // epilogue staging, per softmax warp
+  static constexpr int OFF_BAR = OFF_STG + 8 * STG_WARP;
   static constexpr int WG0 = (BN == 64) ? 2 : 4;     // first softmax warp
   static constexpr int THREADS = 32 * (WG0 + 8);
   static constexpr int CTAS_PER_SM = (BN == 64) ? 2 : 1;
+  // room for aligning the dynamic shared memory base up to 1024 bytes: up to 1 KB, less
+  // when that is what lets CTAS_PER_SM blocks share the SM's 228 KB (1 KB of it reserved
+  // per block); the kernel checks at run time that the slack it needs is there
+  static constexpr int SMEM_CAP = 233472 / CTAS_PER_SM - 1024;
+  static constexpr int SLACK = (SMEM_CAP - (OFF_BAR + 256)) < 1024 ? (SMEM_CAP - (OFF_BAR + 256)) : 1024;
+  static_assert(SLACK >= 0, "shared memory over budget");
+  static_assert(NSTAGE <= 4, "barrier arrays hold 4 stages");
+  static constexpr int SMEM = OFF_BAR + 256 + SLACK;  // + barriers + alignment slack
   static constexpr uint32_t TMEM_COLS = (BN == 64) ? 256 : 512;
   static constexpr uint32_t COL_S = 0;       // + t * BN
   static constexpr uint32_t COL_O = 2 * BN;  // + t * D
@@ -110,6 +130,10 @@ __global__ void __launch_bounds__(FwdCfg<D, BN>::THREADS, FwdCfg<D, BN>::CTAS_PE
   using C = FwdCfg<D, BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  if (smem - smem_raw > C::SLACK) {  // (uniform over the CTA) the buffers would not fit
+    if (threadIdx.x == 0) set_status(FA_ERR_UNSUPPORTED, 62);
+    return;
+  }
   FwdBars* bars = reinterpret_cast<FwdBars*>(smem + C::OFF_BAR);
   volatile int* abort_flag = &bars->abort_flag;
 
@@ -343,6 +367,9 @@ __global__ void __launch_bounds__(FwdCfg<D, BN>::THREADS, FwdCfg<D, BN>::CTAS_PE
         mma_commit(&bars->s_full[0]);
         issue_S(qb, 1, kv % C::NSTAGE);
         mma_commit(&bars->s_full[1]);
+        // the Q buffer is free once the item's last S has been computed (not its last P.V):
+        // the producer then loads the next item's Q while this item's last tile finishes
+        if (n == 1) mma_commit(&bars->q_empty[qb]);
         for (int j = 0; j < n; ++j, ++kv, ++g) {
           const int st = kv % C::NSTAGE;
           const int st2 = (kv + 1) % C::NSTAGE;
@@ -383,9 +410,9 @@ __global__ void __launch_bounds__(FwdCfg<D, BN>::THREADS, FwdCfg<D, BN>::CTAS_PE
           if (more) {
             issue_S(qb, 1, st2);
             mma_commit(&bars->s_full[1]);
+            if (j + 2 == n) mma_commit(&bars->q_empty[qb]);  // that was the item's last S
           } else {
             mma_commit(&bars->o_final[1]);
-            mma_commit(&bars->q_empty[qb]);  // every S of this item has been issued
           }
         }
       }
@@ -517,21 +544,23 @@ __global__ void __launch_bounds__(FwdCfg<D, BN>::THREADS, FwdCfg<D, BN>::CTAS_PE
       if (!ok) break;
       if (idle) continue;
       tc_fence_after();
-      // O = u / l, staged per warp (32 rows x 64 columns, 128-byte swizzle) and written by
-      // a TMA store, which also drops the rows past Nq
+      // O = u / l, staged per warp (32 rows x STG_COLS columns, swizzled as the O map
+      // expects: 128-byte rows with the 128-byte pattern, or 64-byte rows with the 64-byte
+      // one) and written by TMA stores, which also drop the rows past the query rows' end
       const float inv = 1.f / l;
-      uint8_t* stg = smem + C::OFF_STG + (warp - C::WG0) * 4096;
+      uint8_t* stg = smem + C::OFF_STG + (warp - C::WG0) * C::STG_WARP;
       const int row0 = qt * 2 * C::BM + t * C::BM + wq * 32;
 #pragma unroll
-      for (int c = 0; c < D / 64; ++c) {
-        uint32_t o[64];
-        tmem_ld32(tO + c * 64, *reinterpret_cast<uint32_t(*)[32]>(&o[0]));
-        tmem_ld32(tO + c * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&o[32]));
+      for (int c = 0; c < D / C::STG_COLS; ++c) {
+        uint32_t o[C::STG_COLS];
+#pragma unroll
+        for (int h2 = 0; h2 < C::STG_COLS / 32; ++h2)
+          tmem_ld32(tO + c * C::STG_COLS + h2 * 32, *reinterpret_cast<uint32_t(*)[32]>(&o[h2 * 32]));
         tmem_wait_ld();
         if (lane == 0) bulk_wait_read();  // the previous store from this staging buffer
         __syncwarp();
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
+        for (int u = 0; u < C::STG_COLS / 8; ++u) {
           const float2 a = __fmul2_rn(make_float2(__uint_as_float(o[8 * u]), __uint_as_float(o[8 * u + 1])),
                                       make_float2(inv, inv));
           const float2 b2 = __fmul2_rn(make_float2(__uint_as_float(o[8 * u + 2]), __uint_as_float(o[8 * u + 3])),
@@ -540,14 +569,15 @@ __global__ void __launch_bounds__(FwdCfg<D, BN>::THREADS, FwdCfg<D, BN>::CTAS_PE
                                        make_float2(inv, inv));
           const float2 d2 = __fmul2_rn(make_float2(__uint_as_float(o[8 * u + 6]), __uint_as_float(o[8 * u + 7])),
                                        make_float2(inv, inv));
-          *reinterpret_cast<uint4*>(stg + lane * 128 + ((u ^ (lane & 7)) << 4)) =
+          const int chunk = (C::STG_COLS == 64) ? (u ^ (lane & 7)) : (u ^ ((lane >> 1) & 3));
+          *reinterpret_cast<uint4*>(stg + lane * (C::STG_COLS * 2) + (chunk << 4)) =
               make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(b2.x, b2.y), pack_bf16x2(c2.x, c2.y),
                          pack_bf16x2(d2.x, d2.y));
         }
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          tma_store_3d(&tmO, stg, c * 64, row0, bh);
+          tma_store_3d(&tmO, stg, c * C::STG_COLS, row0, bh);
           bulk_commit();
         }
       }

@@ -67,8 +67,9 @@ int fa_version(void);
  * fa_fwd — forward pass.  Writes O (dtype `dtype`) and lse (fp32).
  *   q [B,Hq,Nq,d], k and v [B,Hkv,Nkv,d], o [B,Hq,Nq,d]: dtype `dtype`.
  *   lse [B,Hq,Nq] fp32, may not be NULL.
- *   d in {64, 128}.  dtype BF16: tcgen05 tensor-core kernel, fp32 accumulation, P
- *   rounded to bf16 before P·V.  dtype F32: fp32 SIMT kernel (d == 64 only).
+ *   dtype BF16: d in {64, 96, 128}, tcgen05 tensor-core kernel, fp32 accumulation, P
+ *   rounded to bf16 before P·V (d == 96 runs the d == 128 kernel on zero-filled
+ *   columns).  dtype F32: fp32 SIMT kernel, d == 64.
  *   scale > 0 (usually 1/sqrt(d)); causal 0 or 1.
  * Errors: FA_ERR_INVALID_ARG (null/misaligned pointer, size <= 0, Hq % Hkv != 0,
  * scale not finite or <= 0, causal && Nq > Nkv); FA_ERR_UNSUPPORTED (other d or dtype).
@@ -93,7 +94,8 @@ size_t fa_bwd_workspace_size(int B, int Hq, int Nq, int d);
  *   and dv are summed over the Hq/Hkv query heads that share a key/value head.
  *   workspace: at least fa_bwd_workspace_size(B,Hq,Nq,d) bytes, 256-byte aligned;
  *   its contents on entry do not matter.
- *   d == 64 or 128.
+ *   dtype BF16: d == 64 or 128, tensor-core kernels.  dtype F32: d == 64 and grad_dtype
+ *   F32, CUDA-core kernels (fp32 products throughout).
  * Errors: as fa_fwd, plus FA_ERR_WORKSPACE.
  */
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
@@ -149,7 +151,7 @@ fa_status fa_paged_decode(const void* q, const void* k_cache, const void* v_cach
  *     and every earlier one); 0 = it sees all ctx_lens[r] keys.
  *   o [R,Hq,Nq_max,d] bf16 and lse [R,Hq,Nq_max] fp32 (natural log): rows i >= q_lens[r]
  *     are left undefined (o) or untouched (lse).
- *   d == 64 or 128, block_size == 16, GQA as in fa_fwd.
+ *   d in {64, 96, 128} (as fa_fwd), block_size == 16, GQA as in fa_fwd.
  *   A length or block id out of range is not dereferenced: the kernel skips that request
  *   (or reads block 0 for the bad entry) and sets the device status word
  *   (FA_ERR_INVALID_ARG), so that request's result is undefined.

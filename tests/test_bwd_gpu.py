@@ -81,3 +81,25 @@ def test_bwd_gradient_invariants_on_gpu():
     s_do = do.double().numpy().sum(axis=2)
     assert np.abs(s_dk).max() < 0.05
     assert np.abs(s_dv - s_do).max() < 0.05
+
+
+F32_EDGE = [
+    # B, Hq, Hkv, Nq, Nkv, causal: fp32 inputs take the CUDA-core backward (d = 64)
+    (1, 12, 12, 196, 196, False),  # the fp32 ViT-B/16 layer
+    (1, 1, 1, 1, 1, False),
+    (1, 2, 1, 33, 33, True),
+    (2, 4, 2, 100, 161, False),
+    (1, 3, 1, 70, 300, True),
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Nq,Nkv,causal", F32_EDGE)
+def test_bwd_f32(B, Hq, Hkv, Nq, Nkv, causal):
+    """fp32 gradients against the fp64 oracle at the fp32 bar (max-abs 1e-5), fed the
+    fp32 forward's O and lse as a training step would be."""
+    case = DenseCase("bwd_f32", B, Hq, Hkv, Nq, Nkv, 64, "f32", causal, 90 + Nq + Nkv, 0.125)
+    (q, k, v, do), (dq, dk, dv) = run(case)
+    rq, rk, rv = ora.attention_bwd(q, k, v, do, case.scale, causal)
+    for got, ref, name in ((dq, rq, "dQ"), (dk, rk, "dK"), (dv, rv, "dV")):
+        err = np.abs(to_np(got) - ref).max()
+        assert err <= 1e-5, f"{name}: fp32 max-abs {err:.3e}"

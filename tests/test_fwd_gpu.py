@@ -64,6 +64,8 @@ EDGE = [
     (1, 2, 1, 513, 513, 64, True, "bf16"),
     (1, 8, 2, 1000, 1000, 128, True, "bf16"),
     (1, 2, 1, 1, 300, 128, True, "bf16"),
+    (1, 4, 2, 300, 300, 96, True, "bf16"),
+    (2, 2, 1, 130, 517, 96, False, "bf16"),
     (1, 2, 2, 77, 77, 64, False, "f32"),
     (1, 4, 2, 130, 200, 64, True, "f32"),
     (2, 2, 1, 1, 65, 64, False, "f32"),
@@ -81,6 +83,53 @@ def test_edge_shapes(B, Hq, Hkv, Nq, Nkv, d, causal, dtype):
     else:
         check_bf16(o, O, "O")
         check_lse(lse, L, "lse")
+
+
+# d = 64 with at most 256 keys (the ViT-like regime): ragged key counts inside a 16-key
+# MMA step and a 32-column softmax chunk, query counts spanning several work items
+SHORT = [
+    # B, Hq, Hkv, Nq, Nkv, causal
+    (1, 1, 1, 1, 1, False),
+    (2, 3, 1, 1, 17, False),
+    (1, 2, 2, 15, 15, True),
+    (1, 4, 2, 16, 16, False),
+    (1, 2, 1, 33, 100, True),
+    (2, 4, 4, 196, 196, False),
+    (1, 2, 1, 255, 255, True),
+    (1, 2, 2, 256, 256, False),
+    (1, 3, 3, 300, 256, False),
+    (1, 2, 1, 513, 200, False),
+    (1, 2, 1, 100, 256, True),
+    (3, 2, 2, 600, 17, False),
+    (1, 4, 1, 129, 130, True),
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Nq,Nkv,causal", SHORT)
+def test_short_keys_d64(B, Hq, Hkv, Nq, Nkv, causal):
+    case = DenseCase("short", B, Hq, Hkv, Nq, Nkv, 64, "bf16", causal, 500 + Nq + 3 * Nkv)
+    q, k, v, o, lse = run(case)
+    O, L = ora.attention_fwd(q, k, v, case.scale, causal)
+    check_bf16(o, O, "O")
+    check_lse(lse, L, "lse")
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_short_keys_large_jumps_in_the_row_maximum(causal):
+    """Later keys whose scores exceed the earlier keys' maximum by about 43 and then about
+    100 more (base 2) move the running reference maximum twice; the second jump underflows
+    the earlier terms to zero, as the exact softmax does in fp32."""
+    case = DenseCase("jump", 1, 2, 1, 196, 196, 64, "bf16", causal, 77)
+    q, k, v = case.make()
+    q[..., 0] = 4.0
+    k[0, 0, 70, 0] = 60.0   # scale * q.k = 30 natural units above the rest
+    k[0, 0, 170, 0] = 140.0  # 70 natural units
+    o, lse = fa.fwd(q.cuda(), k.cuda(), v.cuda(), causal=causal, scale=case.scale)
+    torch.cuda.synchronize()
+    assert fa.device_status() == 0
+    O, L = ora.attention_fwd(q, k, v, case.scale, causal)
+    check_bf16(o, O, "O")
+    check_lse(lse, L, "lse")
 
 
 def test_causal_row0_returns_v0_exactly():

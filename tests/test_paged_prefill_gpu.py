@@ -44,6 +44,7 @@ def oracle(inp, causal):
         (128, 8, 8, (129, 640), (128, 100)),
         (64, 6, 2, (300, 65, 777), None),
         (64, 4, 1, (1000, 200, 33), (1000, 1, 7)),
+        (96, 4, 2, (300, 17, 500), (300, 9, 129)),
     ],
 )
 def test_paged_prefill_vs_oracle(d, Hq, Hkv, ctx, ql, causal):
