@@ -72,7 +72,7 @@ def fwd_args(**kw):
         (dict(causal=1, Nq=200, Nkv=100), fa.FA_ERR_INVALID_ARG),
         (dict(q=FAKE + 8), fa.FA_ERR_INVALID_ARG),
         (dict(lse=FAKE + 2), fa.FA_ERR_INVALID_ARG),
-        (dict(d=96), fa.FA_ERR_UNSUPPORTED),
+        (dict(d=80), fa.FA_ERR_UNSUPPORTED),
         (dict(d=128, dtype=fa.FA_DTYPE_F32), fa.FA_ERR_UNSUPPORTED),
         (dict(dtype=7), fa.FA_ERR_UNSUPPORTED),
         (dict(B=70000, Hq=2, Hkv=2), fa.FA_ERR_UNSUPPORTED),
@@ -97,7 +97,8 @@ def bwd_args(**kw):
         (dict(dk=FAKE + 4), fa.FA_ERR_INVALID_ARG),
         (dict(Hq=3), fa.FA_ERR_INVALID_ARG),
         (dict(causal=1, Nq=256), fa.FA_ERR_INVALID_ARG),
-        (dict(dtype=fa.FA_DTYPE_F32), fa.FA_ERR_UNSUPPORTED),
+        (dict(dtype=fa.FA_DTYPE_F32, d=128), fa.FA_ERR_UNSUPPORTED),
+        (dict(dtype=fa.FA_DTYPE_F32, grad_dtype=fa.FA_DTYPE_BF16), fa.FA_ERR_UNSUPPORTED),
         (dict(grad_dtype=9), fa.FA_ERR_UNSUPPORTED),
         (dict(d=256), fa.FA_ERR_UNSUPPORTED),
         (dict(ws=None), fa.FA_ERR_WORKSPACE),
@@ -150,3 +151,30 @@ def test_binding_rejects_cpu_tensors():
     x = torch.zeros(1, 1, 4, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError, match="CUDA"):
         fa.fwd(x, x, x)
+
+
+def pre_args(**kw):
+    a = dict(q=FAKE, kc=FAKE, vc=FAKE, bt=FAKE, ctx=FAKE, ql=FAKE, o=FAKE, lse=FAKE, R=4, Hq=8, Hkv=2, Nq=512,
+             d=128, bs=16, maxb=64, nblocks=100, scale=0.088, causal=1, dtype=fa.FA_DTYPE_BF16, stream=None)
+    a.update(kw)
+    return list(a.values())
+
+
+@pytest.mark.parametrize(
+    "kw,code",
+    [
+        (dict(ql=None), fa.FA_ERR_INVALID_ARG),
+        (dict(lse=None), fa.FA_ERR_INVALID_ARG),
+        (dict(Nq=0), fa.FA_ERR_INVALID_ARG),
+        (dict(Hq=6, Hkv=4), fa.FA_ERR_INVALID_ARG),
+        (dict(causal=3), fa.FA_ERR_INVALID_ARG),
+        (dict(kc=FAKE + 8), fa.FA_ERR_INVALID_ARG),
+        (dict(ctx=FAKE + 2), fa.FA_ERR_INVALID_ARG),
+        (dict(d=80), fa.FA_ERR_UNSUPPORTED),
+        (dict(bs=32), fa.FA_ERR_UNSUPPORTED),
+        (dict(dtype=fa.FA_DTYPE_F32), fa.FA_ERR_UNSUPPORTED),
+        (dict(R=70000), fa.FA_ERR_UNSUPPORTED),
+    ],
+)
+def test_paged_prefill_rejects_on_host(L, kw, code):
+    assert L.fa_paged_prefill(*pre_args(**kw)) == code
