@@ -79,6 +79,7 @@ struct BwdParams {
   void* dk;
   void* dv;
   int grad_bf16;
+  int dout;               // row width of dq, dk, dv and the accumulator (D, or 96 on the D = 128 kernel)
   int Hq, Hkv, Nq, Nkv, Nq_pad;
   float scale;
   float scale_log2;
@@ -128,17 +129,33 @@ __global__ void __launch_bounds__(256) fa_bwd_preprocess_kernel(const __nv_bfloa
     float acc = 0.f;
     if (q < Nq) {
       const size_t base = (size_t(bh) * Nq + q) * D + part * (D / 8);
+      if constexpr ((D / 8) % 8 == 0) {
 #pragma unroll
-      for (int c = 0; c < D / 64; ++c) {
-        const uint4 a = *reinterpret_cast<const uint4*>(o + base + c * 8);
-        const uint4 g = *reinterpret_cast<const uint4*>(dO + base + c * 8);
-        const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
-        const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&g);
+        for (int c = 0; c < D / 64; ++c) {
+          const uint4 a = *reinterpret_cast<const uint4*>(o + base + c * 8);
+          const uint4 g = *reinterpret_cast<const uint4*>(dO + base + c * 8);
+          const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
+          const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&g);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 fa = __bfloat1622float2(a2[e]), fg = __bfloat1622float2(g2[e]);
-          acc = fmaf(fa.x, fg.x, acc);
-          acc = fmaf(fa.y, fg.y, acc);
+          for (int e = 0; e < 4; ++e) {
+            const float2 fa = __bfloat1622float2(a2[e]), fg = __bfloat1622float2(g2[e]);
+            acc = fmaf(fa.x, fg.x, acc);
+            acc = fmaf(fa.y, fg.y, acc);
+          }
+        }
+      } else {  // D = 96: 12 elements per thread, 8-byte loads
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          const uint2 a = *reinterpret_cast<const uint2*>(o + base + c * 4);
+          const uint2 g = *reinterpret_cast<const uint2*>(dO + base + c * 4);
+          const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
+          const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&g);
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const float2 fa = __bfloat1622float2(a2[e]), fg = __bfloat1622float2(g2[e]);
+            acc = fmaf(fa.x, fg.x, acc);
+            acc = fmaf(fa.y, fg.y, acc);
+          }
         }
       }
     }
@@ -440,12 +457,12 @@ __global__ void __launch_bounds__(512, 1)
     // ---- dK_j (half A warps) and dV_j (half B warps); scale already folded into dS
     const uint32_t col = hf == 0 ? C::COL_DK : C::COL_DV;
     void* dst = hf == 0 ? p.dk : p.dv;
-    const size_t base = (size_t(bk) * p.Nkv + key) * D;
+    const size_t base = (size_t(bk) * p.Nkv + key) * p.dout;
     if (ok && n_steps > 0) ok = warp_wait(&bars->dkdv_full, 0, p.wait_ns, abort_flag, 222);
     if (ok && n_steps > 0) {
       tc_fence_after();
 #pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < p.dout / 32; ++c) {
         uint32_t v[32];
         tmem_ld32(tmem + lane_off + col + c * 32, v);
         tmem_wait_ld();
@@ -469,7 +486,7 @@ __global__ void __launch_bounds__(512, 1)
       }
     } else if (n_steps == 0 && key < p.Nkv) {
       // no query row can see these keys: their gradients are zero
-      for (int c = 0; c < D; c += 4) {
+      for (int c = 0; c < p.dout; c += 4) {
         if (p.grad_bf16)
           *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(dst) + base + c) = make_uint2(0, 0);
         else
@@ -513,9 +530,9 @@ __global__ void __launch_bounds__(512, 1)
           bulk_commit();
         }
       } else {
-        float* dstq = p.dq_acc + ((size_t(b) * p.Hq + h) * p.Nq + q) * D;
+        float* dstq = p.dq_acc + ((size_t(b) * p.Hq + h) * p.Nq + q) * p.dout;
 #pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = 0; c < p.dout / 32; ++c) {
           uint32_t v[32];
           tmem_ld32(tmem + lane_off + C::col_dq(qb) + c * 32, v);
           tmem_wait_ld();

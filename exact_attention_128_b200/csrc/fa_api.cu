@@ -150,6 +150,10 @@ fa_status bwd_launch(const void* q, const void* k, const void* v, const void* o,
     fa_bwd_preprocess_kernel<64><<<pre_blocks, 256, 0, st>>>(
         static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, lse2, dstat, dq_acc,
         long(rows_pad), Nq, Nq_pad, long(rows) * d);
+  else if (d == 96)
+    fa_bwd_preprocess_kernel<96><<<pre_blocks, 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, lse2, dstat, dq_acc,
+        long(rows_pad), Nq, Nq_pad, long(rows) * d);
   else
     fa_bwd_preprocess_kernel<128><<<pre_blocks, 256, 0, st>>>(
         static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, lse2, dstat, dq_acc,
@@ -161,7 +165,9 @@ fa_status bwd_launch(const void* q, const void* k, const void* v, const void* o,
       !make_map_bf16(&mv, v, d, Nkv, B * Hkv, 128) || !make_map_bf16(&mo, dO, d, Nq, B * Hq, 128) ||
       !make_map_f32(&mdq, dq_acc, d, Nq, B * Hq))
     return FA_ERR_CUDA;
-  BwdParams prm{dq_acc, lse2, dstat, dk, dv, grad_dtype == FA_DTYPE_BF16 ? 1 : 0, Hq, Hkv, Nq, Nkv, Nq_pad,
+  // d = 96 runs the d = 128 kernel on 96-wide maps (zero-filled columns 96..127); its
+  // gradient rows are written 96 wide
+  BwdParams prm{dq_acc, lse2, dstat, dk, dv, grad_dtype == FA_DTYPE_BF16 ? 1 : 0, d, Hq, Hkv, Nq, Nkv, Nq_pad,
                 scale, scale * 1.4426950408889634f, g_wait_ns};
   fa_status s;
   if (d == 64)
@@ -363,7 +369,7 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   }
   if (dtype != FA_DTYPE_BF16) return FA_ERR_UNSUPPORTED;
   if (grad_dtype != FA_DTYPE_F32 && grad_dtype != FA_DTYPE_BF16) return FA_ERR_UNSUPPORTED;
-  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 96 && d != 128) return FA_ERR_UNSUPPORTED;
   if (long(B) * Hq > 65535) return FA_ERR_UNSUPPORTED;
   const size_t need = fa_bwd_workspace_size(B, Hq, Nq, d);
   if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return FA_ERR_WORKSPACE;

@@ -47,6 +47,8 @@ EDGE = [
     (1, 4, 2, 256, 384, 128, False),
     (1, 3, 1, 100, 612, 64, True),
     (1, 2, 1, 513, 513, 128, True),
+    (1, 4, 2, 200, 200, 96, True),
+    (2, 2, 1, 130, 300, 96, False),
 ]
 
 
