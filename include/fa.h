@@ -67,9 +67,10 @@ int fa_version(void);
  * fa_fwd — forward pass.  Writes O (dtype `dtype`) and lse (fp32).
  *   q [B,Hq,Nq,d], k and v [B,Hkv,Nkv,d], o [B,Hq,Nq,d]: dtype `dtype`.
  *   lse [B,Hq,Nq] fp32, may not be NULL.
- *   dtype BF16: d in {64, 96, 128}, tcgen05 tensor-core kernel, fp32 accumulation, P
- *   rounded to bf16 before P·V (d == 96 runs the d == 128 kernel on zero-filled
- *   columns).  dtype F32: fp32 SIMT kernel, d == 64.
+ *   dtype BF16: d in {64, 96, 128, 256}, tcgen05 tensor-core kernels, fp32 accumulation,
+ *   P rounded to bf16 before P·V (d == 96 runs the d == 128 kernel on zero-filled
+ *   columns; d == 256 has its own one-query-tile kernel).  dtype F32: fp32 SIMT kernel,
+ *   d == 64.
  *   scale > 0 (usually 1/sqrt(d)); causal 0 or 1.
  * Errors: FA_ERR_INVALID_ARG (null/misaligned pointer, size <= 0, Hq % Hkv != 0,
  * scale not finite or <= 0, causal && Nq > Nkv); FA_ERR_UNSUPPORTED (other d or dtype).

@@ -66,6 +66,10 @@ EDGE = [
     (1, 2, 1, 1, 300, 128, True, "bf16"),
     (1, 4, 2, 300, 300, 96, True, "bf16"),
     (2, 2, 1, 130, 517, 96, False, "bf16"),
+    (1, 2, 1, 300, 300, 256, True, "bf16"),
+    (1, 4, 2, 129, 517, 256, False, "bf16"),
+    (2, 2, 2, 1, 70, 256, True, "bf16"),
+    (1, 2, 1, 700, 1000, 256, True, "bf16"),
     (1, 2, 2, 77, 77, 64, False, "f32"),
     (1, 4, 2, 130, 200, 64, True, "f32"),
     (2, 2, 1, 1, 65, 64, False, "f32"),
