@@ -270,7 +270,10 @@ def measure_dense_fwd(case, dev, steps, warmup, world, peaks, peak_key="bf16_tfl
     sec = per_step_ms * 1e-3
     tflops = flops / sec / 1e12
     gbs = nbytes / sec / 1e9
-    kname = f"fa_fwd_bf16_kernel<{case.d},{str(case.causal).lower()}>"
+    if case.d == 256:
+        kname = f"fa_fwd_d256_kernel<{str(case.causal).lower()}>"
+    else:  # d = 96 runs the d = 128 kernel
+        kname = f"fa_fwd_bf16_kernel<{128 if case.d == 96 else case.d},{str(case.causal).lower()}>"
     t_tensor = flops / (peaks[peak_key] * 1e12)
     t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
     if t_hbm > t_tensor:
@@ -287,6 +290,11 @@ def measure_dense_fwd(case, dev, steps, warmup, world, peaks, peak_key="bf16_tfl
                  "hbm_frac": round(gbs / peaks["hbm_gbs"], 4)})
     return {"ms": ms, "per_step_ms": per_step_ms, "tflops": tflops, "roofline": roof, "rot_bytes": rot_bytes,
             "launches_per_step": 1}
+
+
+def fp32_alu_peak_tflops(peaks):
+    """FP32 FFMA peak of the CUDA cores: 148 SMs x 128 lanes x 2 FLOP x max SM clock."""
+    return 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
 
 
 def measure_train(case, dev, steps, warmup, world, peaks):
@@ -317,6 +325,12 @@ def measure_train(case, dev, steps, warmup, world, peaks):
     flops = fwd * 3.5  # forward 2 contractions + backward 5 (score recompute included)
     per = ms / steps
     tflops = flops / (per * 1e-3) / 1e12
+    if case.dtype == "f32":  # CUDA-core FFMA kernels
+        peak = fp32_alu_peak_tflops(peaks)
+        return {"per_step_ms": per, "tflops": tflops,
+                "roofline": {"bound": "alu", "achieved": round(tflops, 3), "peak": round(peak, 1), "unit": "TFLOP/s",
+                             "frac": round(tflops / peak, 4), "peak_kind": "fp32 FFMA, 148 SMs x 128 lanes x 2 x max clock",
+                             "algorithmic_flops_per_step": flops}}
     peak = peaks["bf16_tflops"]
     return {"per_step_ms": per, "tflops": tflops,
             "roofline": {"bound": "tensor", "achieved": round(tflops, 2), "peak": peak, "unit": "TFLOP/s",
@@ -580,7 +594,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--only", choices=["prefill_causal", "prefill_noncausal", "train", "decode", "append", "graph",
-                                       "paged_prefill"],
+                                       "paged_prefill", "d96", "d256", "f32_train"],
                     help="measure just this one secondary workload (for profiling runs) and print it")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -620,6 +634,11 @@ def main():
             r = measure_graph_decode(dev, args.steps, args.warmup, world)
         elif args.only == "paged_prefill":
             r = measure_paged_prefill(W.PAGED_PREFILL, dev, args.steps, args.warmup, world, peaks)
+        elif args.only in ("d96", "d256"):
+            r = measure_dense_fwd(W.D96_PREFILL if args.only == "d96" else W.D256_PREFILL, dev, args.steps,
+                                  args.warmup, world, peaks)
+        elif args.only == "f32_train":
+            r = measure_train(W.VIT_LAYER_F32, dev, args.steps, args.warmup, world, peaks)
         else:
             c = W.GQA_PREFILL_CAUSAL if args.only == "prefill_causal" else W.prefill_sweep()[3]
             r = measure_dense_fwd(c, dev, args.steps, args.warmup, world, peaks)
@@ -658,6 +677,14 @@ def main():
                                               "ms_per_step": round(r["per_step_ms"], 4), "roofline": r["roofline"]}
         except fa.FAError as e:
             secondary[W.TRAIN_CAUSAL.name] = {"unavailable": str(e)}
+        for c in (W.D96_PREFILL, W.D256_PREFILL):
+            torch.cuda.empty_cache()
+            r = measure_dense_fwd(c, dev, 10, 3, world, peaks)
+            secondary[c.name] = {"value": round(r["tflops"], 2), "unit": "TFLOP/s",
+                                 "ms_per_step": round(r["per_step_ms"], 4), "roofline": r["roofline"]}
+        r = measure_train(W.VIT_LAYER_F32, dev, 200, 10, world, peaks)
+        secondary["vit_b16_layer_f32_fwd_bwd"] = {"value": round(r["tflops"], 3), "unit": "TFLOP/s",
+                                                  "ms_per_step": round(r["per_step_ms"], 4), "roofline": r["roofline"]}
         torch.cuda.empty_cache()
         r = measure_paged_prefill(W.PAGED_PREFILL, dev, 20, 5, world, peaks)
         secondary[W.PAGED_PREFILL.name] = {"value": round(r["tflops"], 2), "unit": "TFLOP/s",

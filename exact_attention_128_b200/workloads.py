@@ -84,6 +84,9 @@ VIT_BATCHED_BF16 = DenseCase("vit_b16_batched_fwd_bf16", 64, 12, 12, 196, 196, 6
 GQA_PREFILL_CAUSAL = DenseCase("gqa_prefill_causal_n8192", 4, 32, 8, 8192, 8192, 128, "bf16", True, 3)
 # Training step, causal, 16 heads of d = 64.
 TRAIN_CAUSAL = DenseCase("train_fwd_bwd_causal_n4096", 8, 16, 16, 4096, 4096, 64, "bf16", True, 4, 0.125)
+# Other head dimensions at the prefill sweep's N = 4096 (B*N = 32768 for d = 96).
+D96_PREFILL = DenseCase("d96_prefill_noncausal_n4096", 8, 32, 8, 4096, 4096, 96, "bf16", False, 5)
+D256_PREFILL = DenseCase("d256_prefill_noncausal_n4096", 4, 16, 4, 4096, 4096, 256, "bf16", False, 7)
 
 
 def prefill_sweep():
