@@ -272,8 +272,10 @@ def measure_dense_fwd(case, dev, steps, warmup, world, peaks, peak_key="bf16_tfl
     gbs = nbytes / sec / 1e9
     if case.d == 256:
         kname = f"fa_fwd_d256_kernel<{str(case.causal).lower()}>"
-    else:  # d = 96 runs the d = 128 kernel
-        kname = f"fa_fwd_bf16_kernel<{128 if case.d == 96 else case.d},{str(case.causal).lower()}>"
+    elif case.d == 96:  # the d = 128 kernel on 96-wide rows
+        kname = f"fa_fwd_bf16_kernel<128,{str(case.causal).lower()}>(d=96)"
+    else:
+        kname = f"fa_fwd_bf16_kernel<{case.d},{str(case.causal).lower()}>"
     t_tensor = flops / (peaks[peak_key] * 1e12)
     t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
     if t_hbm > t_tensor:
