@@ -217,7 +217,8 @@ def dense_fwd_step_fns(case, dev, rot=None):
         sets.append((qq, kk, vv, o, lse))
         args = [ctypes.c_void_p(t.data_ptr()) for t in (qq, kk, vv, o, lse)] + [
             case.B, case.Hq, case.Hkv, case.Nq, case.Nkv, case.d, ctypes.c_float(case.scale), int(case.causal),
-            fa.FA_DTYPE_BF16, ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)]
+            fa.FA_DTYPE_F32 if case.dtype == "f32" else fa.FA_DTYPE_BF16,
+            ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)]
 
         def fn(args=args):
             s = L.fa_fwd(*args)
@@ -258,18 +259,28 @@ def measure_dense_fwd(case, dev, steps, warmup, world, peaks, peak_key="bf16_tfl
     """Forward kernel throughput; the roofline is whichever of tensor or HBM binds.
 
     Algorithmic work per launch: 4*d FLOP per allowed (query, key) pair and head; bytes
-    = q, k, v read once + o written once (bf16) + lse (fp32).  The bound is the larger of
-    flops / tensor peak and bytes / HBM peak.
+    = q, k, v read once + o written once + lse (fp32).  The bound is the larger of
+    flops / tensor peak and bytes / HBM peak (fp32 inputs: the CUDA cores' FFMA peak).
     """
     fns, sets, host, rot_bytes = dense_fwd_step_fns(case, dev)
     ms = timed_loop(fns, steps, warmup, world)
     flops = case.fwd_flops()
     q, k, v = host
-    nbytes = 2 * q.numel() * 2 + 2 * k.numel() * 2 + case.B * case.Hq * case.Nq * 4
+    esz = q.element_size()
+    nbytes = 2 * q.numel() * esz + 2 * k.numel() * esz + case.B * case.Hq * case.Nq * 4
     per_step_ms = ms / steps
     sec = per_step_ms * 1e-3
     tflops = flops / sec / 1e12
     gbs = nbytes / sec / 1e9
+    if case.dtype == "f32":
+        kname = "fa_fwd_f32_kernel"
+        peak = fp32_alu_peak_tflops(peaks)
+        roof = {"bound": "alu", "achieved": round(tflops, 3), "peak": round(peak, 1), "unit": "TFLOP/s",
+                "frac": round(tflops / peak, 4), "peak_kind": "fp32 FFMA, 148 SMs x 128 lanes x 2 x max clock",
+                "traffic": None, "kernel": kname, "algorithmic_flops_per_launch": flops,
+                "algorithmic_bytes_per_launch": nbytes, "gbs": round(gbs, 1)}
+        return {"ms": ms, "per_step_ms": per_step_ms, "tflops": tflops, "roofline": roof, "rot_bytes": rot_bytes,
+                "launches_per_step": 1}
     if case.d == 256:
         kname = f"fa_fwd_d256_kernel<{str(case.causal).lower()}>"
     elif case.d == 96:  # the d = 128 kernel on 96-wide rows
@@ -684,6 +695,9 @@ def main():
             r = measure_dense_fwd(c, dev, 10, 3, world, peaks)
             secondary[c.name] = {"value": round(r["tflops"], 2), "unit": "TFLOP/s",
                                  "ms_per_step": round(r["per_step_ms"], 4), "roofline": r["roofline"]}
+        r = measure_dense_fwd(W.VIT_LAYER_F32, dev, 500, 10, world, peaks)
+        secondary[W.VIT_LAYER_F32.name] = {"value": round(r["tflops"], 3), "unit": "TFLOP/s",
+                                           "ms_per_step": round(r["per_step_ms"], 4), "roofline": r["roofline"]}
         r = measure_train(W.VIT_LAYER_F32, dev, 200, 10, world, peaks)
         secondary["vit_b16_layer_f32_fwd_bwd"] = {"value": round(r["tflops"], 3), "unit": "TFLOP/s",
                                                   "ms_per_step": round(r["per_step_ms"], 4), "roofline": r["roofline"]}

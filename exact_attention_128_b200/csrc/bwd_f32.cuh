@@ -13,12 +13,12 @@
 // fp32 inputs need fp32 products, so this path uses FFMA, like the fp32 forward.  Three
 // kernels, no atomics, every result written once:
 //   fa_bwd_f32_pre_kernel   D_i, one warp per query row
-//   fa_bwd_f32_dkdv_kernel  one CTA per (32-key block, batch, kv head): walks the group's
+//   fa_bwd_f32_dkdv_kernel  one CTA per (BR-key block, batch, kv head): walks the group's
 //                           query heads and the query blocks that see the keys
-//   fa_bwd_f32_dq_kernel    one CTA per (32-row query block, batch, query head): walks
+//   fa_bwd_f32_dq_kernel    one CTA per (BR-row query block, batch, query head): walks
 //                           the key blocks the rows see
-// Each step recomputes a 32x32 score tile in shared memory (8 threads per row, 4 scores
-// each) and accumulates 8 output columns per thread.
+// Each step recomputes a BR x BR score tile in shared memory (8 threads per row, BR/8
+// scores each) and accumulates 8 output columns per thread; the library launches BR = 32.
 #pragma once
 #include "common.cuh"
 
@@ -26,11 +26,7 @@ namespace fa {
 
 namespace b32 {
 constexpr int D = 64;
-constexpr int BQ = 32;        // query rows per block
-constexpr int BK = 32;        // keys per block
-constexpr int THREADS = 256;  // 8 threads per row of a 32-row tile
-constexpr int RP = D + 1;     // padded row of a [32 x 64] tile
-constexpr int SP = BK + 1;    // padded row of a [32 x 32] tile
+constexpr int RP = D + 1;  // padded row of a [BR x 64] tile
 }  // namespace b32
 
 struct BwdF32Params {
@@ -64,38 +60,43 @@ __global__ void __launch_bounds__(256) fa_bwd_f32_pre_kernel(const float* o, con
 
 namespace b32 {
 
-// rows [r0, r0 + 32) of a [n, 64] matrix into a padded tile; rows past n read as zero
+// rows [r0, r0 + BR) of a [n, 64] matrix into a padded tile; rows past n read as zero
+template <int BR>
 __device__ __forceinline__ void load_tile(float (*dst)[RP], const float* src, int r0, int n) {
-  for (int e = threadIdx.x; e < 32 * D; e += THREADS) {
+  for (int e = threadIdx.x; e < BR * D; e += 8 * BR) {
     const int r = e / D, c = e % D;
     dst[r][c] = (r0 + r < n) ? src[size_t(r0 + r) * D + c] : 0.f;
   }
 }
 
-// the 4 dot products a[i] . b[j0 + u], u < 4, of 64-long rows
-__device__ __forceinline__ void dot4(const float (*a)[RP], const float (*b)[RP], int i, int j0, float (&out)[4]) {
+// the N dot products a[i] . b[j0 + u], u < N, of 64-long rows
+template <int N>
+__device__ __forceinline__ void dotn(const float (*a)[RP], const float (*b)[RP], int i, int j0, float (&out)[N]) {
 #pragma unroll
-  for (int u = 0; u < 4; ++u) out[u] = 0.f;
+  for (int u = 0; u < N; ++u) out[u] = 0.f;
 #pragma unroll 16
   for (int c = 0; c < D; ++c) {
     const float x = a[i][c];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) out[u] = fmaf(x, b[j0 + u][c], out[u]);
+    for (int u = 0; u < N; ++u) out[u] = fmaf(x, b[j0 + u][c], out[u]);
   }
 }
 
-// P and dS of one 32x32 tile: rows qi0 + i (query), columns kj0 + j (key); thread owns
-// row i = tid / 8 and columns j0 .. j0 + 3, j0 = (tid % 8) * 4.
+// P and dS of one BR x BR tile: rows qi0 + i (query), columns kj0 + j (key); thread owns
+// row i = tid / 8 and columns j0 .. j0 + BR/8 - 1, j0 = (tid % 8) * BR/8.
+template <int BR>
 __device__ __forceinline__ void p_ds_tile(const float (*sQ)[RP], const float (*sK)[RP], const float (*sdO)[RP],
-                                          const float (*sV)[RP], const float* sL, const float* sD, float (*sP)[SP],
-                                          float (*sS)[SP], int qi0, int kj0, const BwdF32Params& p) {
-  const int i = threadIdx.x >> 3, j0 = (threadIdx.x & 7) * 4;
-  float s[4], dp[4];
-  dot4(sQ, sK, i, j0, s);
-  dot4(sdO, sV, i, j0, dp);
+                                          const float (*sV)[RP], const float* sL, const float* sD,
+                                          float (*sP)[BR + 1], float (*sS)[BR + 1], int qi0, int kj0,
+                                          const BwdF32Params& p) {
+  constexpr int N = BR / 8;
+  const int i = threadIdx.x >> 3, j0 = (threadIdx.x & 7) * N;
+  float s[N], dp[N];
+  dotn<N>(sQ, sK, i, j0, s);
+  dotn<N>(sdO, sV, i, j0, dp);
   const int qi = qi0 + i, off = p.Nkv - p.Nq;
 #pragma unroll
-  for (int u = 0; u < 4; ++u) {
+  for (int u = 0; u < N; ++u) {
     const int kj = kj0 + j0 + u;
     const bool ok = qi < p.Nq && kj < p.Nkv && (!p.causal || kj <= qi + off);
     const float pij = ok ? expf(s[u] * p.scale - sL[i]) : 0.f;
@@ -106,15 +107,17 @@ __device__ __forceinline__ void p_ds_tile(const float (*sQ)[RP], const float (*s
 
 }  // namespace b32
 
-__global__ void __launch_bounds__(b32::THREADS) fa_bwd_f32_dkdv_kernel(const BwdF32Params p) {
+template <int BR>
+__global__ void __launch_bounds__(8 * BR) fa_bwd_f32_dkdv_kernel(const BwdF32Params p) {
   using namespace b32;
+  constexpr int BQ = BR, BK = BR;
   __shared__ float sK[BK][RP], sV[BK][RP], sQ[BQ][RP], sdO[BQ][RP];
-  __shared__ float sP[BQ][SP], sS[BQ][SP], sL[BQ], sD[BQ];
+  __shared__ float sP[BQ][BR + 1], sS[BQ][BR + 1], sL[BQ], sD[BQ];
   const int kb = blockIdx.x, bk = blockIdx.y;  // key block; batch * Hkv + kv head
   const int b = bk / p.Hkv, hk = bk % p.Hkv, G = p.Hq / p.Hkv;
   const int kj0 = kb * BK;
-  load_tile(sK, p.k + size_t(bk) * p.Nkv * D, kj0, p.Nkv);
-  load_tile(sV, p.v + size_t(bk) * p.Nkv * D, kj0, p.Nkv);
+  load_tile<BR>(sK, p.k + size_t(bk) * p.Nkv * D, kj0, p.Nkv);
+  load_tile<BR>(sV, p.v + size_t(bk) * p.Nkv * D, kj0, p.Nkv);
   // thread owns key j = tid / 8, columns c0 .. c0 + 7
   const int j = threadIdx.x >> 3, c0 = (threadIdx.x & 7) * 8;
   float adk[8], adv[8];
@@ -128,15 +131,15 @@ __global__ void __launch_bounds__(b32::THREADS) fa_bwd_f32_dkdv_kernel(const Bwd
     for (int qb = qb0; qb * BQ < p.Nq; ++qb) {
       const int qi0 = qb * BQ;
       __syncthreads();  // the previous step's tiles are consumed
-      load_tile(sQ, p.q + bh * p.Nq * D, qi0, p.Nq);
-      load_tile(sdO, p.dO + bh * p.Nq * D, qi0, p.Nq);
+      load_tile<BR>(sQ, p.q + bh * p.Nq * D, qi0, p.Nq);
+      load_tile<BR>(sdO, p.dO + bh * p.Nq * D, qi0, p.Nq);
       if (threadIdx.x < BQ) {
         const int qi = qi0 + threadIdx.x;
         sL[threadIdx.x] = qi < p.Nq ? p.lse[bh * p.Nq + qi] : 0.f;
         sD[threadIdx.x] = qi < p.Nq ? p.Dvec[bh * p.Nq + qi] : 0.f;
       }
       __syncthreads();
-      p_ds_tile(sQ, sK, sdO, sV, sL, sD, sP, sS, qi0, kj0, p);
+      p_ds_tile<BR>(sQ, sK, sdO, sV, sL, sD, sP, sS, qi0, kj0, p);
       __syncthreads();
 #pragma unroll 4
       for (int i = 0; i < BQ; ++i) {
@@ -161,16 +164,18 @@ __global__ void __launch_bounds__(b32::THREADS) fa_bwd_f32_dkdv_kernel(const Bwd
   }
 }
 
-__global__ void __launch_bounds__(b32::THREADS) fa_bwd_f32_dq_kernel(const BwdF32Params p) {
+template <int BR>
+__global__ void __launch_bounds__(8 * BR) fa_bwd_f32_dq_kernel(const BwdF32Params p) {
   using namespace b32;
+  constexpr int BQ = BR, BK = BR;
   __shared__ float sK[BK][RP], sV[BK][RP], sQ[BQ][RP], sdO[BQ][RP];
-  __shared__ float sP[BQ][SP], sS[BQ][SP], sL[BQ], sD[BQ];
+  __shared__ float sP[BQ][BR + 1], sS[BQ][BR + 1], sL[BQ], sD[BQ];
   const int qb = blockIdx.x, bh = blockIdx.y;  // query block; batch * Hq + head
   const int b = bh / p.Hq, h = bh % p.Hq;
   const size_t bk = size_t(b) * p.Hkv + h / (p.Hq / p.Hkv);
   const int qi0 = qb * BQ;
-  load_tile(sQ, p.q + size_t(bh) * p.Nq * D, qi0, p.Nq);
-  load_tile(sdO, p.dO + size_t(bh) * p.Nq * D, qi0, p.Nq);
+  load_tile<BR>(sQ, p.q + size_t(bh) * p.Nq * D, qi0, p.Nq);
+  load_tile<BR>(sdO, p.dO + size_t(bh) * p.Nq * D, qi0, p.Nq);
   if (threadIdx.x < BQ) {
     const int qi = qi0 + threadIdx.x;
     sL[threadIdx.x] = qi < p.Nq ? p.lse[size_t(bh) * p.Nq + qi] : 0.f;
@@ -185,10 +190,10 @@ __global__ void __launch_bounds__(b32::THREADS) fa_bwd_f32_dq_kernel(const BwdF3
   const int kv_end = p.causal ? min(p.Nkv, qi0 + BQ + (p.Nkv - p.Nq)) : p.Nkv;
   for (int kj0 = 0; kj0 < kv_end; kj0 += BK) {
     __syncthreads();  // the previous step's tiles are consumed (and this block's Q, dO loaded)
-    load_tile(sK, p.k + bk * p.Nkv * D, kj0, p.Nkv);
-    load_tile(sV, p.v + bk * p.Nkv * D, kj0, p.Nkv);
+    load_tile<BR>(sK, p.k + bk * p.Nkv * D, kj0, p.Nkv);
+    load_tile<BR>(sV, p.v + bk * p.Nkv * D, kj0, p.Nkv);
     __syncthreads();
-    p_ds_tile(sQ, sK, sdO, sV, sL, sD, sP, sS, qi0, kj0, p);
+    p_ds_tile<BR>(sQ, sK, sdO, sV, sL, sD, sP, sS, qi0, kj0, p);
     __syncthreads();
 #pragma unroll 4
     for (int jj = 0; jj < BK; ++jj) {

@@ -16,9 +16,9 @@ namespace fa {
 
 namespace f32 {
 constexpr int D = 64;
-constexpr int BQ = 64;        // query rows per CTA
+constexpr int BQ = 64;        // query rows per CTA (16 when 64-row CTAs would not fill the GPU)
 constexpr int BK = 32;        // keys per tile
-constexpr int THREADS = 256;  // 4 threads per query row
+constexpr int THREADS = 256;  // 4 threads per query row (4 * BQ)
 constexpr int KPAD = D + 1;   // padded K row (bank-conflict free score loop)
 constexpr int PPAD = BK + 1;  // padded P row
 }  // namespace f32
@@ -34,8 +34,13 @@ struct FwdF32Params {
   int causal;
 };
 
-__global__ void __launch_bounds__(f32::THREADS) fa_fwd_f32_kernel(const FwdF32Params p) {
-  using namespace f32;
+template <int BQ>
+__global__ void __launch_bounds__(4 * BQ) fa_fwd_f32_kernel(const FwdF32Params p) {
+  using f32::D;
+  using f32::BK;
+  using f32::KPAD;
+  using f32::PPAD;
+  constexpr int THREADS = 4 * BQ;
   __shared__ float Ks[BK * KPAD];
   __shared__ __align__(16) float Vs[BK * D];
   __shared__ float Ps[BQ * PPAD];

@@ -92,6 +92,7 @@ F32_EDGE = [
     (1, 2, 1, 33, 33, True),
     (2, 4, 2, 100, 161, False),
     (1, 3, 1, 70, 300, True),
+    (4, 8, 8, 320, 320, True),
 ]
 
 

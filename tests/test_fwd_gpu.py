@@ -73,6 +73,7 @@ EDGE = [
     (1, 2, 2, 77, 77, 64, False, "f32"),
     (1, 4, 2, 130, 200, 64, True, "f32"),
     (2, 2, 1, 1, 65, 64, False, "f32"),
+    (4, 16, 4, 320, 320, 64, True, "f32"),  # enough rows for the 64-row variant
 ]
 
 
