@@ -25,6 +25,7 @@ import hashlib
 import json
 import math
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -50,12 +51,17 @@ def load_peaks():
 
 
 def kernel_sources_sha(files) -> str:
-    """Hash of the kernel source files a profile was taken on (csrc-relative names)."""
+    """Hash of the code (comments and layout stripped) of the kernel source files a
+    profile was taken on (csrc-relative names): any change to the code voids the stored
+    traffic figure, a comment edit does not."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "exact_attention_128_b200", "csrc")
     for f in sorted(files):
-        with open(os.path.join(csrc, f), "rb") as fh:
-            h.update(f.encode() + fh.read())
+        with open(os.path.join(csrc, f), encoding="utf-8") as fh:
+            text = fh.read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", " ", text)
+        h.update(f.encode() + " ".join(text.split()).encode())
     return h.hexdigest()[:16]
 
 

@@ -21,9 +21,16 @@
 //               (bf16) over S_t in TMEM, rescales u_t in TMEM when m rose, and at the
 //               end of an item writes O = u/l and lse.
 // While one warpgroup runs the softmax of its tile, the tensor core works on the
-// other tile, so the exponentials overlap the MMAs.
+// other tile, so the exponentials overlap the MMAs.  The Q buffer is released when an
+// item's last S has been computed, so the next item's Q loads during its last tile.
 //
-// TMEM columns (512 allocated): S0 [0,128), S1 [128,256), u0 [256,256+D), u1 after.
+// PAGED (fa_paged_prefill): the same roles over a paged KV cache.  Each request has its
+// own key count and query-row count (its last positions); the producer warp gathers the
+// K/V tiles block by block through the block table ("Atención tipo FlashAttention y
+// atención paginada", the-ai.news).
+//
+// TMEM columns (d = 128, 512 allocated): S0 [0,128), S1 [128,256), u0 [256,256+D), u1
+// after; d = 64 (256 allocated, two CTAs per SM): S0, S1, u0, u1 of 64 columns each.
 // Shared memory: QBUF x (Q0, Q1), then NSTAGE K tiles and NSTAGE V tiles, each stored
 // as D/64 column blocks of [rows x 128 bytes] with the 128-byte swizzle TMA writes and
 // the MMA descriptors expect.
