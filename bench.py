@@ -38,6 +38,7 @@ METRIC = "attention TFLOP/s & % of B200 BF16 tensor peak; paged-decode HBM GB/s"
 L2_BYTES = 126 * 2**20
 NOMINAL_BF16_TFLOPS = 2250.0
 NOMINAL_HBM_GBS = 8000.0
+EX2_PER_CLK_SM = 16  # SFU ex2.approx.f32 throughput per SM per clock (microbenchmark on B200)
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -307,6 +308,12 @@ def measure_dense_fwd(case, dev, steps, warmup, world, peaks, peak_key="bf16_tfl
                  "algorithmic_bytes_per_launch": nbytes, "tflops": round(tflops, 2), "gbs": round(gbs, 1),
                  "tensor_frac": round(tflops / peaks[peak_key], 4),
                  "hbm_frac": round(gbs / peaks["hbm_gbs"], 4)})
+    # secondary ceiling: one exponential per allowed (query, key) pair and head on the SFU,
+    # at 16 ex2 per clock per SM (measured on this GPU) and the maximum SM clock
+    exps = case.B * case.Hq * case.allowed_pairs()
+    exp_s = exps / (EX2_PER_CLK_SM * 148 * peaks.get("sm_max_mhz", 1965.0) * 1e6)
+    roof["exp_bound"] = {"tflops": round(flops / exp_s / 1e12, 1), "frac": round(exp_s / sec, 4),
+                         "ex2_per_launch": exps}
     return {"ms": ms, "per_step_ms": per_step_ms, "tflops": tflops, "roofline": roof, "rot_bytes": rot_bytes,
             "launches_per_step": 1}
 
