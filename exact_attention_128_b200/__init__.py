@@ -7,7 +7,13 @@ call is rejected, an exception is raised.
 
     o, lse = fwd(q, k, v, causal=False)             # q [B,Hq,N,d], k/v [B,Hkv,N,d]
     dq, dk, dv = bwd(q, k, v, o, lse, do, causal=False)
+    paged_kv_append(k_new, v_new, k_cache, v_cache, block_table, positions)
     o, lse = paged_decode(q, k_cache, v_cache, block_table, ctx_lens)
+    o, lse = paged_prefill(q, k_cache, v_cache, block_table, ctx_lens, q_lens, causal=True)
+
+bf16 inputs run on the tensor cores (d in {64, 96, 128, 256} forward, {64, 96, 128}
+backward); fp32 inputs (d = 64) on the CUDA cores.  Paged caches are
+[num_blocks, Hkv, 16, d].
 """
 from __future__ import annotations
 
