@@ -236,29 +236,86 @@ def dense_fwd_step_fns(case, dev, rot=None):
     return fns, sets, (q, k, v), rot * set_bytes
 
 
-def e2e_fwd(case, dev, steps, warmup, world):
-    """Same metric through the public API with pinned host buffers: H2D q,k,v, fwd, D2H o,lse."""
+def e2e_fwd(case, dev, steps, warmup, world, pipelined=True):
+    """Same metric through the public API with pinned host buffers: every step copies its
+    q, k, v host -> device, runs the forward, and reads o and lse back device -> host.
+
+    pipelined: the copies in, the forward and the read-back run on three streams with two
+    device buffer sets, so step i+1's inputs cross PCIe while step i computes and returns
+    its result (each step still moves all of its bytes).  Otherwise every step is serial
+    on one stream.
+    """
     import torch
 
     import exact_attention_128_b200 as fa
 
     q, k, v = (t.pin_memory() for t in case.make())
-    qd, kd, vd = torch.empty_like(q, device=dev), torch.empty_like(k, device=dev), torch.empty_like(v, device=dev)
-    oh = torch.empty_like(q).pin_memory()
-    lh = torch.empty(case.B, case.Hq, case.Nq, dtype=torch.float32).pin_memory()
-    od, ld = torch.empty_like(qd), torch.empty(case.B, case.Hq, case.Nq, device=dev, dtype=torch.float32)
+    nb = 2 if pipelined else 1
+    dev_in = [tuple(torch.empty_like(t, device=dev) for t in (q, k, v)) for _ in range(nb)]
+    dev_out = [(torch.empty_like(dev_in[0][0]),
+                torch.empty(case.B, case.Hq, case.Nq, device=dev, dtype=torch.float32)) for _ in range(nb)]
+    host_out = [(torch.empty_like(q).pin_memory(), torch.empty(case.B, case.Hq, case.Nq, dtype=torch.float32).pin_memory())
+                for _ in range(nb)]
+    main = torch.cuda.current_stream()
+    s_in, s_comp, s_out = (torch.cuda.Stream(device=dev) for _ in range(3)) if pipelined else (main, main, main)
+    ev_in = [torch.cuda.Event() for _ in range(nb)]
+    ev_comp = [torch.cuda.Event() for _ in range(nb)]
+    ev_out = [torch.cuda.Event() for _ in range(nb)]
+    used = [False] * nb
+    i_step = [0]
 
     def step():
-        qd.copy_(q, non_blocking=True)
-        kd.copy_(k, non_blocking=True)
-        vd.copy_(v, non_blocking=True)
-        fa.fwd(qd, kd, vd, causal=case.causal, scale=case.scale, out=od, lse=ld)
-        oh.copy_(od, non_blocking=True)
-        lh.copy_(ld, non_blocking=True)
+        b = i_step[0] % nb
+        i_step[0] += 1
+        qd, kd, vd = dev_in[b]
+        od, ld = dev_out[b]
+        oh, lh = host_out[b]
+        with torch.cuda.stream(s_in):
+            if used[b]:
+                s_in.wait_event(ev_comp[b])  # the forward that read these inputs is done
+            qd.copy_(q, non_blocking=True)
+            kd.copy_(k, non_blocking=True)
+            vd.copy_(v, non_blocking=True)
+            ev_in[b].record(s_in)
+        with torch.cuda.stream(s_comp):
+            s_comp.wait_event(ev_in[b])
+            if used[b]:
+                s_comp.wait_event(ev_out[b])  # the previous read-back of these outputs is done
+            fa.fwd(qd, kd, vd, causal=case.causal, scale=case.scale, out=od, lse=ld)
+            ev_comp[b].record(s_comp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_comp[b])
+            oh.copy_(od, non_blocking=True)
+            lh.copy_(ld, non_blocking=True)
+            ev_out[b].record(s_out)
+        used[b] = True
 
-    ms = timed_loop([step], steps, warmup, world)
+    def join():  # the timed region ends when every stream's work has finished
+        if pipelined:
+            for st in (s_in, s_comp, s_out):
+                main.wait_stream(st)
+
+    for _ in range(warmup):
+        step()
+    join()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(main)
+    if pipelined:
+        for st in (s_in, s_comp, s_out):
+            st.wait_stream(main)
+    for _ in range(steps):
+        step()
+    join()
+    e1.record(main)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), world)
     h2d = sum(t.numel() * t.element_size() for t in (q, k, v))
-    d2h = oh.numel() * oh.element_size() + lh.numel() * 4
+    d2h = host_out[0][0].numel() * host_out[0][0].element_size() + host_out[0][1].numel() * 4
     return ms, h2d, d2h
 
 
@@ -688,10 +745,13 @@ def main():
     e2e = None
     if not args.no_e2e:
         e_steps = max(3, min(args.steps, 200))
-        ms, h2d, d2h = e2e_fwd(case, dev, e_steps, args.warmup, world)
+        ms, h2d, d2h = e2e_fwd(case, dev, e_steps, args.warmup, world, pipelined=True)
+        ms_serial, _, _ = e2e_fwd(case, dev, e_steps, args.warmup, world, pipelined=False)
         e2e = {"value": round(world * case.fwd_flops() * e_steps / (ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e_steps,
-               "ms_per_step": round(ms / e_steps, 4)}
+               "ms_per_step": round(ms / e_steps, 4),
+               "schedule": "copy-in, forward and read-back of consecutive steps overlap on three streams",
+               "serial_ms_per_step": round(ms_serial / e_steps, 4)}
 
     secondary = {}
     if not args.no_secondary and world == 1:
