@@ -45,6 +45,9 @@ def oracle(inp, causal):
         (64, 6, 2, (300, 65, 777), None),
         (64, 4, 1, (1000, 200, 33), (1000, 1, 7)),
         (96, 4, 2, (300, 17, 500), (300, 9, 129)),
+        # whole cache blocks, but a partial key tile: no slot tail, blocks past the sequence
+        (128, 4, 2, (96, 160, 16), None),
+        (64, 4, 2, (48, 96, 208), (48, 3, 100)),
     ],
 )
 def test_paged_prefill_vs_oracle(d, Hq, Hkv, ctx, ql, causal):
