@@ -627,6 +627,24 @@ def cpu_oracle_dense(case, budget_s=12.0):
                       f"{dt:.1f} s, NumPy fp64 materialising the score matrix"}
 
 
+def cpu_oracle_one_head(case, train=False):
+    """The fp64 oracle on one whole (b, h) head of a long workload (forward, or forward +
+    backward), extrapolated linearly to all B*Hq heads: a reported baseline, labelled so."""
+    from oracle import attention_fp64 as ora
+
+    t = case.make(with_grad_output=train)
+    q, k, v = (ora.to_f64(x[0, 0]) for x in t[:3])
+    t0 = time.perf_counter()
+    ora.attention_head(q, k, v, case.scale, case.causal)
+    if train:
+        ora.attention_bwd_head(q, k, v, ora.to_f64(t[3][0, 0]), case.scale, case.causal)
+    dt = time.perf_counter() - t0
+    heads = case.B * case.Hq
+    flops = case.fwd_flops() * (3.5 if train else 1.0)
+    return {"value": flops / (dt * heads) / 1e12, "unit": "TFLOP/s", "cores": oracle_threads(), "kind": "oracle",
+            "sample": f"1 whole (b,h) head of {case.name} in {dt:.2f} s, extrapolated to {heads} heads"}
+
+
 def reference_line(case, args):
     """The oracle as the reference arm: W + K steps, each step whole heads of the workload.
 
@@ -767,11 +785,16 @@ def main():
             r = measure_dense_fwd(c, dev, 20, 5, world, peaks)
             secondary[c.name] = {"value": round(r["tflops"], 2), "unit": "TFLOP/s",
                                  "ms_per_step": round(r["per_step_ms"], 4), "roofline": r["roofline"]}
+            if not args.no_cpu_baseline:
+                secondary[c.name]["cpu_oracle_extrapolated"] = cpu_oracle_one_head(c)
             torch.cuda.empty_cache()
         try:
             r = measure_train(W.TRAIN_CAUSAL, dev, 10, 3, world, peaks)
             secondary[W.TRAIN_CAUSAL.name] = {"value": round(r["tflops"], 2), "unit": "TFLOP/s",
                                               "ms_per_step": round(r["per_step_ms"], 4), "roofline": r["roofline"]}
+            if not args.no_cpu_baseline:
+                secondary[W.TRAIN_CAUSAL.name]["cpu_oracle_extrapolated"] = cpu_oracle_one_head(W.TRAIN_CAUSAL,
+                                                                                               train=True)
         except fa.FAError as e:
             secondary[W.TRAIN_CAUSAL.name] = {"unavailable": str(e)}
         for c in (W.D96_PREFILL, W.D256_PREFILL):
