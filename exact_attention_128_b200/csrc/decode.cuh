@@ -11,9 +11,9 @@
 //
 // Work split (split-KV): CTA (split s, kv head g, request r) covers logical blocks
 // [s*CHUNK, (s+1)*CHUNK) of request r (CHUNK = 128 blocks = 2048 tokens by default).  Each
-// of its 4 warps takes every 4th block and
-// keeps its own (m, l, u) state; the warps' states and then the splits' partial
-// results are merged by weighting each part with its unnormalised mass e^{lse_s}
+// of its 4 warps takes every 4th block and keeps its own (m, l, u) state; the warps'
+// states and then the splits' partial results are merged by weighting each part with
+// its unnormalised mass e^{lse_s}
 // ("No basta con promediar los resultados de los bloques": block results are never
 // simply averaged).  A request that fits in one split writes its output directly.
 //
