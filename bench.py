@@ -10,10 +10,14 @@ total size exceeds twice the L2 cache, bracketed by a barrier and a device
 synchronisation, timed with CUDA events on the launching stream.  Under torchrun
 each rank runs its own replica (weak scaling) and the slowest rank's time counts.
 
-The headline workload is the batched ViT-B/16 attention layer (B=64, H=12, N=196,
-d=64, bf16 forward).  With secondary measurements on (the default at one GPU) the
-line also carries the long causal GQA prefill, the non-causal N=8192 prefill, the
-causal training step (forward + backward) and the paged decode step.
+The headline workload is the largest single-GPU forward: the non-causal GQA prefill at
+N=16384 (B=2, Hq=32, Hkv=8, d=128, bf16; 8.8 TFLOP per call), the end point of the
+sweep over N at B*N = 32768.  With secondary measurements on (the default at one GPU)
+the line ends with a compact record of every other workload: the other sweep points,
+the long causal GQA prefill, the causal training step (forward + backward), the paged
+decode step, the batched ViT-B/16 layer, the paged prefill, head dimensions 96 and 256,
+the fp32 ViT layer (forward; forward + backward), the KV-cache append and the CUDA-graph
+decode step.  Their full records go to stderr.
 
 `--impl reference` times the fp64 CPU oracle on a bounded sample of the same
 workload (the only other implementation of this method here).
@@ -605,109 +609,196 @@ def oracle_threads():
     return len(os.sched_getaffinity(0))
 
 
+class OracleRows:
+    """The fp64 oracle over a dense workload in units of up to `rows` query rows of one
+    (b, h) head (whole heads when N <= rows), each unit one call of its exact per-row
+    forward function on that head's stored values (so no N x N fp64 matrix larger than
+    rows x Nkv is ever held).  Counts the algorithmic FLOPs of the rows done."""
+
+    def __init__(self, case, rows=2048):
+        self.case = case
+        self.q, self.k, self.v = case.make()
+        self.rows = min(rows, case.Nq)
+        self.per_head = (case.Nq + self.rows - 1) // self.rows
+        self.units = case.B * case.Hq * self.per_head
+        self.G = case.Hq // case.Hkv
+        self.done = 0
+        self.flops = 0.0
+        self.rows_done = 0
+
+    def step(self):
+        from oracle import attention_fp64 as ora
+
+        c = self.case
+        u = self.done % self.units
+        bh, part = divmod(u, self.per_head)
+        b, h = divmod(bh, c.Hq)
+        r0 = part * self.rows
+        rows = list(range(r0, min(c.Nq, r0 + self.rows)))
+        g = h // self.G
+        ora.attention_fwd_rows(self.q[b:b + 1, h:h + 1], self.k[b:b + 1, g:g + 1], self.v[b:b + 1, g:g + 1],
+                               c.scale, c.causal, 0, 0, rows)
+        off = c.Nkv - c.Nq
+        keys = sum(min(c.Nkv, i + off + 1) for i in rows) if c.causal else len(rows) * c.Nkv
+        self.flops += 4.0 * c.d * keys
+        self.rows_done += len(rows)
+        self.done += 1
+
+    def describe(self):
+        return (f"{self.done} unit(s) of <= {self.rows} query rows of one (b,h) head of {self.case.name} "
+                f"({self.rows_done} rows, {self.rows_done / (self.case.B * self.case.Hq * self.case.Nq):.4f} of "
+                f"the workload), NumPy fp64 materialising each unit's score rows")
+
+
 def cpu_oracle_dense(case, budget_s=12.0):
-    """Time the fp64 oracle on whole heads of the workload until ~budget_s of CPU work."""
-    import numpy as np
-
-    from oracle import attention_fp64 as ora
-
-    q, k, v = case.make()
-    qn, kn, vn = (ora.to_f64(t) for t in (q, k, v))
-    G = case.Hq // case.Hkv
-    heads = [(b, h) for b in range(case.B) for h in range(case.Hq)]
-    done, t0 = 0, time.perf_counter()
-    while time.perf_counter() - t0 < budget_s:
-        b, h = heads[done % len(heads)]
-        ora.attention_head(qn[b, h], kn[b, h // G], vn[b, h // G], case.scale, case.causal)
-        done += 1
+    """Time the fp64 oracle on units of the workload until ~budget_s of CPU work."""
+    orc = OracleRows(case)
+    t0 = time.perf_counter()
+    while orc.done == 0 or time.perf_counter() - t0 < budget_s:
+        orc.step()
     dt = time.perf_counter() - t0
-    flops = case.fwd_flops() / len(heads) * done
-    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": oracle_threads(), "kind": "oracle",
-            "sample": f"{done} whole (b,h) heads of {case.name} ({done / len(heads):.2f} passes), "
-                      f"{dt:.1f} s, NumPy fp64 materialising the score matrix"}
+    return {"value": orc.flops / dt / 1e12, "unit": "TFLOP/s", "cores": oracle_threads(), "kind": "oracle",
+            "sample": orc.describe() + f", {dt:.1f} s"}
 
 
-def cpu_oracle_one_head(case, train=False):
-    """The fp64 oracle on one whole (b, h) head of a long workload (forward, or forward +
-    backward), extrapolated linearly to all B*Hq heads: a reported baseline, labelled so."""
+def cpu_oracle_extrapolated(case, train=False, budget_s=2.0):
+    """The fp64 oracle on a bounded sample of a long workload, reported as a rate (which
+    is what a linear extrapolation to the whole workload gives): forward row units, or
+    one whole (b, h) head forward + backward for a training step."""
     from oracle import attention_fp64 as ora
 
-    t = case.make(with_grad_output=train)
-    q, k, v = (ora.to_f64(x[0, 0]) for x in t[:3])
+    if not train:
+        r = cpu_oracle_dense(case, budget_s)
+        r["sample"] += ", extrapolated to the whole workload"
+        return r
+    t = case.make(with_grad_output=True)
+    q, k, v, do = (ora.to_f64(x[0, 0]) for x in t)
     t0 = time.perf_counter()
     ora.attention_head(q, k, v, case.scale, case.causal)
-    if train:
-        ora.attention_bwd_head(q, k, v, ora.to_f64(t[3][0, 0]), case.scale, case.causal)
+    ora.attention_bwd_head(q, k, v, do, case.scale, case.causal)
     dt = time.perf_counter() - t0
     heads = case.B * case.Hq
-    flops = case.fwd_flops() * (3.5 if train else 1.0)
-    return {"value": flops / (dt * heads) / 1e12, "unit": "TFLOP/s", "cores": oracle_threads(), "kind": "oracle",
-            "sample": f"1 whole (b,h) head of {case.name} in {dt:.2f} s, extrapolated to {heads} heads"}
+    return {"value": case.fwd_flops() * 3.5 / (dt * heads) / 1e12, "unit": "TFLOP/s", "cores": oracle_threads(),
+            "kind": "oracle", "sample": f"1 whole (b,h) head of {case.name} forward + backward in {dt:.2f} s, "
+                                        f"extrapolated to {heads} heads"}
 
 
 def reference_line(case, args):
-    """The oracle as the reference arm: W + K steps, each step whole heads of the workload.
-
-    Heads per step are sized from one probe head so the whole run stays within
-    ``args.reference_seconds`` (90 s by default).
-    """
-    from oracle import attention_fp64 as ora
-
-    q, k, v = case.make()
-    qn, kn, vn = (ora.to_f64(t) for t in (q, k, v))
-    G = case.Hq // case.Hkv
-    heads = [(b, h) for b in range(case.B) for h in range(case.Hq)]
+    """The oracle as the reference arm: W + K steps, each step the same number of row units
+    of the workload, sized from one probe unit so the whole run stays within
+    ``args.reference_seconds`` (90 s by default)."""
+    orc = OracleRows(case)
     t0 = time.perf_counter()
-    ora.attention_head(qn[0, 0], kn[0, 0], vn[0, 0], case.scale, case.causal)
-    t_head = max(time.perf_counter() - t0, 1e-4)
-    per_step = max(1, min(len(heads), int(args.reference_seconds / ((args.steps + args.warmup) * t_head))))
-    idx = 0
+    orc.step()
+    t_unit = max(time.perf_counter() - t0, 1e-4)
+    per_step = max(1, min(orc.units, int(args.reference_seconds / ((args.steps + args.warmup) * t_unit))))
 
     def step():
-        nonlocal idx
         for _ in range(per_step):
-            b, h = heads[idx % len(heads)]
-            idx += 1
-            ora.attention_head(qn[b, h], kn[b, h // G], vn[b, h // G], case.scale, case.causal)
+            orc.step()
 
     for _ in range(args.warmup):
         step()
+    f0, r0 = orc.flops, orc.rows_done
     t0 = time.perf_counter()
     for _ in range(args.steps):
         step()
     dt = time.perf_counter() - t0
-    flops = case.fwd_flops() / len(heads) * per_step * args.steps
-    value = flops / dt / 1e12
+    value = (orc.flops - f0) / dt / 1e12
+    rows = orc.rows_done - r0
     cb = {"value": value, "unit": "TFLOP/s", "cores": oracle_threads(), "kind": "oracle",
-          "sample": f"{per_step} whole (b,h) head(s) of {case.name} per step, {args.steps} steps, {dt:.1f} s"}
+          "sample": f"{per_step} unit(s) of <= {orc.rows} query rows of one (b,h) head of {case.name} per step "
+                    f"({rows} rows over {args.steps} steps), {dt:.1f} s"}
     # under torchrun with N ranks the job is N-wide, but rank 0 alone times the oracle
     return {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
             "config": {"workload": case.name, "B": case.B, "Hq": case.Hq, "Hkv": case.Hkv, "N": case.Nq,
-                       "d": case.d, "causal": case.causal, "sample_heads_per_step": per_step,
+                       "d": case.d, "causal": case.causal, "sample_units_per_step": per_step,
                        "parallelism": "rank 0 on its host cores" + (f" (of {args.gpus} ranks)" if args.gpus > 1 else "")},
             "cpu_baseline": cb,
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def compact(r, value_key, digits=2):
+    """[value, unit, ms per step, roofline frac, DRAM traffic / algorithmic bytes or None]."""
+    roof = r.get("roofline", {})
+    tr = roof.get("traffic")
+    alg = roof.get("algorithmic_bytes_per_launch")
+    ratio = round(tr / alg, 2) if tr and alg else None
+    unit = "GB/s" if value_key == "gbs" else "TFLOP/s"
+    return [round(r[value_key], digits), unit, round(r["per_step_ms"], 4), roof.get("frac"), ratio]
+
+
 # ----------------------------------------------------------------------------- main
+HEADLINE = "gqa_prefill_noncausal_n16384"
+
+
+def run_secondaries(W, case, dev, world, peaks, no_cpu):
+    """Every other workload, each timed over >= 50 steps (300 for the microsecond ones).
+
+    Returns (compact, detail): compact[name] = [value, unit, ms per step, roofline frac,
+    DRAM traffic / algorithmic bytes]; detail[name] = the full measurement."""
+    import torch
+
+    import exact_attention_128_b200 as fa
+
+    compact_out, detail = {}, {}
+
+    def put(name, r, key, digits=2, oracle=None):
+        compact_out[name] = compact(r, key, digits)
+        r = {k: v for k, v in r.items() if k != "rot_bytes"}
+        if oracle is not None:
+            r["cpu_oracle_extrapolated"] = oracle
+            compact_out[name].append(round(oracle["value"], 4))
+        detail[name] = r
+        torch.cuda.empty_cache()
+
+    for c in (*W.prefill_sweep(), W.GQA_PREFILL_CAUSAL):
+        if c.name == case.name:
+            continue
+        r = measure_dense_fwd(c, dev, 50, 5, world, peaks)
+        put(c.name, r, "tflops", oracle=None if no_cpu else cpu_oracle_extrapolated(c))
+    try:
+        r = measure_train(W.TRAIN_CAUSAL, dev, 50, 5, world, peaks)
+        put(W.TRAIN_CAUSAL.name, r, "tflops",
+            oracle=None if no_cpu else cpu_oracle_extrapolated(W.TRAIN_CAUSAL, train=True))
+    except fa.FAError as e:
+        compact_out[W.TRAIN_CAUSAL.name] = detail[W.TRAIN_CAUSAL.name] = {"unavailable": str(e)}
+    r = measure_decode(W.PAGED_DECODE, dev, 300, 10, world, peaks)
+    put(W.PAGED_DECODE.name, r, "gbs", 1)
+    if case.name != W.VIT_BATCHED_BF16.name:
+        put(W.VIT_BATCHED_BF16.name, measure_dense_fwd(W.VIT_BATCHED_BF16, dev, 300, 10, world, peaks), "tflops")
+    put(W.PAGED_PREFILL.name, measure_paged_prefill(W.PAGED_PREFILL, dev, 50, 5, world, peaks), "tflops")
+    for c in (W.D96_PREFILL, W.D256_PREFILL):
+        put(c.name, measure_dense_fwd(c, dev, 50, 5, world, peaks), "tflops")
+    put(W.VIT_LAYER_F32.name, measure_dense_fwd(W.VIT_LAYER_F32, dev, 300, 10, world, peaks), "tflops", 3)
+    put("vit_b16_layer_f32_fwd_bwd", measure_train(W.VIT_LAYER_F32, dev, 300, 10, world, peaks), "tflops", 3)
+    put("paged_kv_append_r64_hkv2_d128", measure_append(W.PAGED_DECODE, dev, 300, 10, world, peaks), "gbs", 2)
+    g = measure_graph_decode(dev, 300, 10, world)
+    compact_out["graph_decode_r8_append_plus_decode"] = [g["eager_ms_per_step"], g["graph_ms_per_step"]]
+    detail["graph_decode_r8_append_plus_decode"] = g
+    return compact_out, detail
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10000)
-    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="vit_b16_batched_fwd_bf16")
+    ap.add_argument("--workload", default=HEADLINE)
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--reference-seconds", type=float, default=90.0,
                     help="--impl reference: host-time budget of the whole oracle run")
     ap.add_argument("--only", choices=["prefill_causal", "prefill_noncausal", "train", "decode", "append", "graph",
-                                       "paged_prefill", "d96", "d256", "f32_train"],
+                                       "paged_prefill", "d96", "d256", "f32_train", "vit"],
                     help="measure just this one secondary workload (for profiling runs) and print it")
+    ap.add_argument("--decode-split", type=int, default=0,
+                    help="cache blocks per decode split (0: the library's default)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -734,6 +825,8 @@ def main():
     dev = torch.device("cuda", local)
     fa.lib()
     fa.device_status(reset=True)
+    if args.decode_split:
+        fa.set_decode_split(args.decode_split)
 
     if args.only:
         if args.only == "train":
@@ -751,9 +844,12 @@ def main():
                                   args.warmup, world, peaks)
         elif args.only == "f32_train":
             r = measure_train(W.VIT_LAYER_F32, dev, args.steps, args.warmup, world, peaks)
+        elif args.only == "vit":
+            r = measure_dense_fwd(W.VIT_BATCHED_BF16, dev, args.steps, args.warmup, world, peaks)
+        elif args.only == "prefill_causal":
+            r = measure_dense_fwd(W.GQA_PREFILL_CAUSAL, dev, args.steps, args.warmup, world, peaks)
         else:
-            c = W.GQA_PREFILL_CAUSAL if args.only == "prefill_causal" else W.prefill_sweep()[3]
-            r = measure_dense_fwd(c, dev, args.steps, args.warmup, world, peaks)
+            r = measure_dense_fwd(case, dev, args.steps, args.warmup, world, peaks)
         r.pop("rot_bytes", None)
         if rank == 0:
             print(json.dumps({"only": args.only, "steps": args.steps, **r}))
@@ -768,7 +864,7 @@ def main():
 
     e2e = None
     if not args.no_e2e:
-        e_steps = max(3, min(args.steps, 200))
+        e_steps = max(3, min(args.steps, 50))
         ms, h2d, d2h = e2e_fwd(case, dev, e_steps, args.warmup, world, pipelined=True)
         ms_serial, _, _ = e2e_fwd(case, dev, e_steps, args.warmup, world, pipelined=False)
         e2e = {"value": round(world * case.fwd_flops() * e_steps / (ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
@@ -776,51 +872,16 @@ def main():
                "ms_per_step": round(ms / e_steps, 4),
                "schedule": "copy-in, forward and read-back of consecutive steps overlap on three streams",
                "serial_ms_per_step": round(ms_serial / e_steps, 4)}
+    torch.cuda.empty_cache()
 
-    secondary = {}
+    secondary, sec_clocks = {}, None
     if not args.no_secondary and world == 1:
-        for c in (W.GQA_PREFILL_CAUSAL, W.prefill_sweep()[3]):
-            if c.name == case.name:
-                continue
-            r = measure_dense_fwd(c, dev, 20, 5, world, peaks)
-            secondary[c.name] = {"value": round(r["tflops"], 2), "unit": "TFLOP/s",
-                                 "ms_per_step": round(r["per_step_ms"], 4), "roofline": r["roofline"]}
-            if not args.no_cpu_baseline:
-                secondary[c.name]["cpu_oracle_extrapolated"] = cpu_oracle_one_head(c)
-            torch.cuda.empty_cache()
-        try:
-            r = measure_train(W.TRAIN_CAUSAL, dev, 10, 3, world, peaks)
-            secondary[W.TRAIN_CAUSAL.name] = {"value": round(r["tflops"], 2), "unit": "TFLOP/s",
-                                              "ms_per_step": round(r["per_step_ms"], 4), "roofline": r["roofline"]}
-            if not args.no_cpu_baseline:
-                secondary[W.TRAIN_CAUSAL.name]["cpu_oracle_extrapolated"] = cpu_oracle_one_head(W.TRAIN_CAUSAL,
-                                                                                               train=True)
-        except fa.FAError as e:
-            secondary[W.TRAIN_CAUSAL.name] = {"unavailable": str(e)}
-        for c in (W.D96_PREFILL, W.D256_PREFILL):
-            torch.cuda.empty_cache()
-            r = measure_dense_fwd(c, dev, 10, 3, world, peaks)
-            secondary[c.name] = {"value": round(r["tflops"], 2), "unit": "TFLOP/s",
-                                 "ms_per_step": round(r["per_step_ms"], 4), "roofline": r["roofline"]}
-        r = measure_dense_fwd(W.VIT_LAYER_F32, dev, 500, 10, world, peaks)
-        secondary[W.VIT_LAYER_F32.name] = {"value": round(r["tflops"], 3), "unit": "TFLOP/s",
-                                           "ms_per_step": round(r["per_step_ms"], 4), "roofline": r["roofline"]}
-        r = measure_train(W.VIT_LAYER_F32, dev, 200, 10, world, peaks)
-        secondary["vit_b16_layer_f32_fwd_bwd"] = {"value": round(r["tflops"], 3), "unit": "TFLOP/s",
-                                                  "ms_per_step": round(r["per_step_ms"], 4), "roofline": r["roofline"]}
-        torch.cuda.empty_cache()
-        r = measure_paged_prefill(W.PAGED_PREFILL, dev, 20, 5, world, peaks)
-        secondary[W.PAGED_PREFILL.name] = {"value": round(r["tflops"], 2), "unit": "TFLOP/s",
-                                           "ms_per_step": round(r["per_step_ms"], 4), "roofline": r["roofline"]}
-        torch.cuda.empty_cache()
-        r = measure_decode(W.PAGED_DECODE, dev, 300, 10, world, peaks)
-        secondary[W.PAGED_DECODE.name] = {"value": round(r["gbs"], 1), "unit": "GB/s",
-                                          "ms_per_step": round(r["per_step_ms"], 5), "roofline": r["roofline"]}
-        secondary["graph_decode_r8_append_plus_decode"] = measure_graph_decode(dev, 300, 10, world)
-        r = measure_append(W.PAGED_DECODE, dev, 300, 10, world, peaks)
-        secondary["paged_kv_append_r64_hkv2_d128"] = {"value": round(r["gbs"], 2), "unit": "GB/s",
-                                                      "ms_per_step": round(r["per_step_ms"], 5),
-                                                      "roofline": r["roofline"]}
+        sampler2 = ClockSampler(local)
+        sampler2.start()
+        secondary, detail = run_secondaries(W, case, dev, world, peaks, args.no_cpu_baseline)
+        sec_clocks = sampler2.stop()
+        # the full secondary records go to stderr; stdout keeps the one JSON line
+        print("secondary detail: " + json.dumps(detail), file=sys.stderr)
 
     status = fa.device_status(reset=True)
     if status != 0:
@@ -853,8 +914,13 @@ def main():
         "e2e": e2e,
         "gpu_launches": head["launches_per_step"] * args.steps,
         "clocks": clocks,
-        "secondary": secondary,
     }
+    if secondary:
+        # last, so that a reader keeping only the end of the line still sees every workload:
+        # name: [value, unit, ms/step, roofline frac, DRAM traffic / algorithmic bytes (null:
+        # no profile of the current code), fp64 oracle TFLOP/s where timed]
+        line["secondary_clocks"] = {k: sec_clocks[k] for k in ("sm_mhz", "reasons")} if sec_clocks else None
+        line["secondary"] = secondary
     if rank == 0:
         print(json.dumps(line))
     if world > 1:

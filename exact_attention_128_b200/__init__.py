@@ -34,6 +34,7 @@ __all__ = [
     "paged_kv_append",
     "paged_prefill",
     "device_status",
+    "set_decode_split",
     "set_wait_limit_ns",
     "selftest_wait_timeout",
     "EXPORTED",
@@ -63,7 +64,7 @@ EXPORTED = {
     "fa_device_status": (_i, [_i]),
     "fa_set_wait_limit_ns": (None, [ctypes.c_uint64]),
     "fa_selftest_wait_timeout": (_i, [_vp]),
-    "fa_selftest_exp2": (_i, [_vp, _vp, _i, _vp]),
+    "fa_set_decode_split": (_i, [_i]),
 }
 
 
@@ -250,6 +251,14 @@ def paged_prefill(q, k_cache, v_cache, block_table, ctx_lens, q_lens, causal: bo
 
 def device_status(reset: bool = True) -> int:
     return int(lib().fa_device_status(int(bool(reset))))
+
+
+def set_decode_split(blocks: int) -> int:
+    """Cache blocks per decode split (multiple of 4 in [32, 128]; 0 = default); returns the old value."""
+    old = int(lib().fa_set_decode_split(int(blocks)))
+    if old < 0:
+        raise ValueError(f"decode split of {blocks} blocks is out of range")
+    return old
 
 
 def set_wait_limit_ns(ns: int):

@@ -92,6 +92,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64
   }
 }
 
+// Bounded wait that ignores the abort flag and records nothing: for draining loads that
+// are still in flight after an abort.  Returns false if `limit_ns` elapsed first.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity))
+    if (globaltimer_ns() - t0 > limit_ns) return false;
+  return true;
+}
+
 // Every lane of the warp waits; the warp proceeds only if all lanes saw the phase
 // complete, so the .sync.aligned tcgen05 instructions that follow stay convergent.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
@@ -261,30 +270,6 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
-}
-
-// 2^x on the FMA pipe for a pair of values, x <= 0, used alongside the SFU so the
-// exponentials of a softmax tile are split over two execution pipes.  Range reduction
-// after Cody and Waite: x = j + f with j = round-to-nearest(x) (by adding and subtracting
-// 1.5 * 2^23) and f in [-1/2, 1/2]; 2^f by a degree-4 polynomial whose coefficients were
-// fitted for this library (iterated weighted least squares on Chebyshev nodes, relative
-// error <= 2.7e-6 on [-1/2, 1/2] in fp32 Horner form); j is added to the exponent bits.
-// Inputs below -126 are clamped, so results are >= 2^-126 rather than 0: callers use it
-// only where no score is masked.
-__device__ __forceinline__ float2 exp2_fma2(float2 x) {
-  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
-  x.x = fmaxf(x.x, -126.0f);
-  x.y = fmaxf(x.y, -126.0f);
-  const float2 t = __fadd2_rn(x, make_float2(kRound, kRound));
-  const float2 j = __fadd2_rn(t, make_float2(-kRound, -kRound));
-  const float2 f = __fadd2_rn(x, make_float2(-j.x, -j.y));
-  float2 q = __ffma2_rn(make_float2(0.009570100344717503f, 0.009570100344717503f), f,
-                        make_float2(0.05591786280274391f, 0.05591786280274391f));
-  q = __ffma2_rn(q, f, make_float2(0.240247443318367f, 0.240247443318367f));
-  q = __ffma2_rn(q, f, make_float2(0.6931217908859253f, 0.6931217908859253f));
-  q = __ffma2_rn(q, f, make_float2(0.9999992847442627f, 0.9999992847442627f));
-  return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23)),
-                     __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
 }
 
 // max(a, b, c) in one instruction (sm_100 three-input max).

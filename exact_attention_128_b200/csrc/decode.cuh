@@ -10,8 +10,9 @@
 // ("Mecanismo y detalles", GQA) are processed together, so each K/V byte is read once.
 //
 // Work split (split-KV): CTA (split s, kv head g, request r) covers logical blocks
-// [s*CHUNK, (s+1)*CHUNK) of request r (CHUNK = 128 blocks = 2048 tokens by default).  Each
-// of its 4 warps takes every 4th block and keeps its own (m, l, u) state; the warps'
+// [s*chunk, (s+1)*chunk) of request r; the host picks chunk (a multiple of 4 blocks, at
+// most MAX_CHUNK = 128 blocks = 2048 tokens) per call.  Each of its 4 warps takes every
+// 4th block and keeps its own (m, l, u) state; the warps'
 // states and then the splits' partial results are merged by weighting each part with
 // its unnormalised mass e^{lse_s}
 // ("No basta con promediar los resultados de los bloques": block results are never
@@ -33,13 +34,11 @@ constexpr int BS = 16;          // tokens per cache block
 #ifndef FA_DEC_STAGES
 #define FA_DEC_STAGES 2
 #endif
-#ifndef FA_DEC_CHUNK
-#define FA_DEC_CHUNK 128
-#endif
 constexpr int WARPS = 4;
 constexpr int STAGES = FA_DEC_STAGES;  // blocks in flight per warp
-constexpr int CHUNK = FA_DEC_CHUNK;    // logical blocks per CTA (split size = CHUNK * 16 tokens)
-static_assert(CHUNK / WARPS <= 32, "a warp's block-table entries are held one per lane");
+constexpr int MAX_CHUNK = 128;         // largest split, in logical blocks (2048 tokens)
+constexpr int MIN_CHUNK = 32;          // smallest split the host may choose (workspace sizing)
+static_assert(MAX_CHUNK / WARPS <= 32, "a warp's block-table entries are held one per lane");
 constexpr int SLAB = BS * D * 2;  // 4096 bytes: one (block, kv head) slab of K or V
 constexpr int STAGE_BYTES = 2 * SLAB;
 constexpr int OFF_BAR = WARPS * STAGES * STAGE_BYTES;
@@ -58,6 +57,7 @@ struct DecodeParams {
   float* part_o;
   float* part_lse;
   int R, Hq, Hkv, max_blocks, num_blocks, max_splits;
+  int chunk;  // logical blocks per split: a multiple of WARPS, at most MAX_CHUNK
   float scale_log2;
   uint64_t wait_ns;
 };
@@ -103,13 +103,13 @@ __global__ void __launch_bounds__(dec::WARPS * 32)
     return;
   }
   const int nblk = (ctx + BS - 1) / BS;
-  const int nsplit = (nblk + CHUNK - 1) / CHUNK;
-  const int b0 = s * CHUNK;
+  const int nsplit = (nblk + p.chunk - 1) / p.chunk;
+  const int b0 = s * p.chunk;
   if (b0 >= nblk) {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     return;
   }
-  const int b1 = min(nblk, b0 + CHUNK);
+  const int b1 = min(nblk, b0 + p.chunk);
 
   const int warp = warp_id(), lane = lane_id();
   const int gq = lane >> 2;  // mma group id: query-head row, key token, output column
@@ -124,7 +124,7 @@ __global__ void __launch_bounds__(dec::WARPS * 32)
   fence_barrier_init();
   __syncthreads();
 
-  // physical block of this warp's i-th block, held by lane i (CHUNK / WARPS <= 32)
+  // physical block of this warp's i-th block, held by lane i (chunk / WARPS <= 32)
   int my_phys = 0;
   if (lane < nb) {
     my_phys = p.bt[size_t(r) * p.max_blocks + b0 + warp + lane * WARPS];
@@ -177,9 +177,11 @@ __global__ void __launch_bounds__(dec::WARPS * 32)
   const int v_tok = rr + 8 * (mi & 1), v_chunk_hi = mi >> 1;  // V: (token, n-tile parity)
 
   bool ok = true;
+  int consumed = 0;  // stages this warp has waited for (loads issued: min(nb, consumed + STAGES))
   for (int i = 0; i < nb && ok; ++i) {
     ok = warp_wait(&bars[i % STAGES], (i / STAGES) & 1, p.wait_ns, &abort_flag, 102);
     if (!ok) break;
+    consumed = i + 1;
     const uint32_t sk = sbase + (i % STAGES) * STAGE_BYTES;
     const uint32_t sv = sk + SLAB;
     const int lb = b0 + warp + i * WARPS;
@@ -256,13 +258,36 @@ __global__ void __launch_bounds__(dec::WARPS * 32)
     }
   }
 
+  if (!ok) {
+    // A bounded wait ran out (here or in another warp): let this warp's loads that are
+    // still in flight land before the CTA gives up its shared memory, each wait again
+    // bounded (and no longer cut short by the abort flag).
+    if (lane == 0)
+      for (int i = consumed; i < min(nb, consumed + STAGES); ++i)
+        mbar_wait_bounded(&bars[i % STAGES], (i / STAGES) & 1, p.wait_ns);
+    __syncwarp();
+  }
+
   // ---- merge the warps' (m, l, u) states
   l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
   l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
   l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
   l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
   __syncthreads();  // all warps done with their stages: reuse shared memory
-  if (abort_flag) return;
+  if (abort_flag) {
+    // the device status word already says FA_ERR_DEVICE_TIMEOUT; mark this split's result
+    // as NaN so neither the output nor the merge of the other splits looks valid
+    for (int idx = threadIdx.x; idx < G * D; idx += WARPS * 32) {
+      const int h = g * G + idx / D, d = idx % D;
+      if (nsplit == 1) {
+        p.o[(size_t(r) * p.Hq + h) * D + d] = __float2bfloat16_rn(NAN);
+        if (d == 0 && p.lse) p.lse[size_t(r) * p.Hq + h] = NAN;
+      } else if (d == 0) {
+        p.part_lse[(size_t(r) * p.Hq + h) * p.max_splits + s] = NAN;
+      }
+    }
+    return;
+  }
   float* so = reinterpret_cast<float*>(dsmem);  // [WARPS][MAX_G][OP]
   float* sm = so + WARPS * MAX_G * OP;          // [WARPS][MAX_G]
   float* sl = sm + WARPS * MAX_G;               // [WARPS][MAX_G]
@@ -346,11 +371,20 @@ __global__ void __launch_bounds__(128) fa_paged_decode_combine_kernel(const Deco
   const int r = rh / p.Hq;
   const int ctx = p.ctx[r];
   if (ctx < 1 || ctx > p.max_blocks * BS) return;
-  const int nsplit = ((ctx + BS - 1) / BS + CHUNK - 1) / CHUNK;
+  const int nsplit = ((ctx + BS - 1) / BS + p.chunk - 1) / p.chunk;
   if (nsplit <= 1) return;
   const float* pl = p.part_lse + size_t(rh) * p.max_splits;
   float M = -INFINITY;
-  for (int s = 0; s < nsplit; ++s) M = fmaxf(M, pl[s]);
+  bool aborted = false;  // a split whose bounded wait ran out left NaN
+  for (int s = 0; s < nsplit; ++s) {
+    M = fmaxf(M, pl[s]);
+    aborted |= isnan(pl[s]);
+  }
+  if (aborted) {
+    p.o[size_t(rh) * D + threadIdx.x] = __float2bfloat16_rn(NAN);
+    if (threadIdx.x == 0 && p.lse) p.lse[rh] = NAN;
+    return;
+  }
   float W = 0.f, U = 0.f;
   const int d = threadIdx.x;
   for (int s = 0; s < nsplit; ++s) {

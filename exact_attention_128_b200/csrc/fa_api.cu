@@ -28,6 +28,17 @@ using namespace fa;
 
 uint64_t g_wait_ns = 200000000ull;  // 200 ms per wait
 
+// Logical blocks per decode split; 0 = the library's choice (kDecodeChunk).
+#ifndef FA_DEC_CHUNK
+#define FA_DEC_CHUNK 128
+#endif
+constexpr int kDecodeChunk = FA_DEC_CHUNK;
+static_assert(kDecodeChunk >= fa::dec::MIN_CHUNK && kDecodeChunk <= fa::dec::MAX_CHUNK &&
+                  kDecodeChunk % fa::dec::WARPS == 0, "decode split size out of range");
+int g_dec_chunk = 0;
+int decode_chunk() { return g_dec_chunk > 0 ? g_dec_chunk : kDecodeChunk; }
+int decode_splits(int max_blocks) { return (max_blocks + decode_chunk() - 1) / decode_chunk(); }
+
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -190,17 +201,6 @@ fa_status bwd_launch(const void* q, const void* k, const void* v, const void* o,
   return FA_OK;
 }
 
-__global__ void selftest_exp2_kernel(const float* x, float* y, int n) {
-  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
-  if (i + 1 < n) {
-    const float2 r = exp2_fma2(make_float2(x[i], x[i + 1]));
-    y[i] = r.x;
-    y[i + 1] = r.y;
-  } else if (i < n) {
-    y[i] = exp2_fma2(make_float2(x[i], x[i])).x;
-  }
-}
-
 __global__ void selftest_wait_kernel(uint64_t limit_ns) {
   __shared__ uint64_t bar;
   __shared__ int abort_flag;
@@ -246,13 +246,6 @@ fa_status fa_device_status(int reset) {
 
 fa_status fa_selftest_wait_timeout(void* stream) {
   selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(g_wait_ns);
-  return launched();
-}
-
-fa_status fa_selftest_exp2(const float* x, float* y, int n, void* stream) {
-  if (!x || !y || n <= 0) return FA_ERR_INVALID_ARG;
-  const int pairs = (n + 1) / 2;
-  selftest_exp2_kernel<<<(pairs + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
   return launched();
 }
 
@@ -424,8 +417,15 @@ fa_status fa_paged_kv_append(const void* k_new, const void* v_new, void* k_cache
 
 size_t fa_paged_decode_workspace_size(int R, int Hq, int d, int max_blocks_per_seq, int block_size) {
   if (R <= 0 || Hq <= 0 || d <= 0 || max_blocks_per_seq <= 0 || block_size <= 0) return 0;
-  const size_t splits = size_t((max_blocks_per_seq + dec::CHUNK - 1) / dec::CHUNK);
+  const size_t splits = size_t(decode_splits(max_blocks_per_seq));
   return align256(size_t(R) * Hq * splits * d * sizeof(float)) + align256(size_t(R) * Hq * splits * sizeof(float));
+}
+
+int fa_set_decode_split(int blocks) {
+  if (blocks != 0 && (blocks < dec::MIN_CHUNK || blocks > dec::MAX_CHUNK || blocks % dec::WARPS != 0)) return -1;
+  const int old = g_dec_chunk;
+  g_dec_chunk = blocks;
+  return old;
 }
 
 fa_status fa_paged_decode(const void* q, const void* k_cache, const void* v_cache, const int* block_table,
@@ -444,12 +444,13 @@ fa_status fa_paged_decode(const void* q, const void* k_cache, const void* v_cach
   if (Hq / Hkv > dec::MAX_G || R > 65535 || Hkv > 65535) return FA_ERR_UNSUPPORTED;
   const size_t need = fa_paged_decode_workspace_size(R, Hq, d, max_blocks_per_seq, block_size);
   if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return FA_ERR_WORKSPACE;
-  const int max_splits = (max_blocks_per_seq + dec::CHUNK - 1) / dec::CHUNK;
+  const int chunk = decode_chunk();
+  const int max_splits = decode_splits(max_blocks_per_seq);
   float* part_o = static_cast<float*>(workspace);
   float* part_lse =
       reinterpret_cast<float*>(static_cast<char*>(workspace) + align256(size_t(R) * Hq * max_splits * d * 4));
   DecodeParams prm{static_cast<const __nv_bfloat16*>(q), block_table, ctx_lens, static_cast<__nv_bfloat16*>(o),
-                   lse, part_o, part_lse, R, Hq, Hkv, max_blocks_per_seq, num_blocks, max_splits,
+                   lse, part_o, part_lse, R, Hq, Hkv, max_blocks_per_seq, num_blocks, max_splits, chunk,
                    scale * 1.4426950408889634f, g_wait_ns};
   CUtensorMap mk, mv;
   const long cache_rows = long(num_blocks) * Hkv * dec::BS;
@@ -492,22 +493,57 @@ namespace {
 static __device__ __align__(256) unsigned char g_noalloc_scratch[FA_NOALLOC_SCRATCH_BYTES];
 
 constexpr int kMaxDevices = 64;
-void* g_noalloc_ptr[kMaxDevices] = {};
+struct ScratchAddr {
+  unsigned long long ctx_id;  // CUDA context the address belongs to (unique per context)
+  void* ptr;
+};
+ScratchAddr g_noalloc_addr[kMaxDevices] = {};
 std::mutex g_noalloc_mu;
 
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// Unique id of the calling thread's current CUDA context (0 if it cannot be had).  A
+// context that is destroyed and re-created (cudaDeviceReset) gets a new id, and its copy
+// of the library's device image a new address.
+unsigned long long current_ctx_id() {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
 // Device address of the scratch array on the current device.  In host code the array's
-// name is only a host-side stand-in, so the address is looked up once per device with
-// that device current, and cached.
+// name is only a host-side stand-in, so the address is looked up with
+// cudaGetSymbolAddress, with the device current, on the first call in each CUDA context of
+// the device (once per device, unless its context is reset), and cached.
 fa_status noalloc_scratch(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
+  ScratchAddr& a = g_noalloc_addr[dev];
+  const unsigned long long id = current_ctx_id();
+  if (!a.ptr || id == 0 || id != a.ctx_id) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return FA_ERR_CUDA;
-    g_noalloc_ptr[dev] = p;
+    a.ptr = p;
+    a.ctx_id = id != 0 ? id : current_ctx_id();  // the lookup may have made the context current
   }
-  *out = g_noalloc_ptr[dev];
+  *out = a.ptr;
   return FA_OK;
 }
 

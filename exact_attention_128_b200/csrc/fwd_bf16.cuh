@@ -39,15 +39,6 @@
 
 namespace fa {
 
-// Bit k set: in unmasked tiles, element pair k of every 8 pairs takes the FMA-pipe
-// exponential (exp2_fma2) instead of the SFU one.  Off by default: measured on B200 with
-// 0x24, 0xA4, 0xAA and 0xB6 (25-50 %), every split was slower than the SFU alone in this
-// kernel (e.g. 1006 vs 845-930 TFLOP/s at N = 8192, d = 128), because the softmax warps
-// are limited by issue slots and latency, not by SFU throughput.
-#ifndef FWD_EMU_PAIRS
-#define FWD_EMU_PAIRS 0x00u
-#endif
-
 // Lazy rescaling threshold (base-2 units) for the running reference maximum; see the
 // softmax loop.  8 keeps every P <= 256, far inside bf16 and fp32 range.
 #ifndef FA_RESCALE_LOG2
@@ -507,14 +498,14 @@ __global__ void __launch_bounds__(FwdCfg<D, BN>::THREADS, FwdCfg<D, BN>::CTAS_PE
               tmem_st16(tS + c * 16, pk);
             }
           } else {
-            // interior tile: pairs FWD_EMU_PAIRS of every 8 take the FMA-pipe exponential
+            // interior tile: no masked column
 #pragma unroll
             for (int c = 0; c < C::BN / 32; ++c) {
               uint32_t pk[16];
 #pragma unroll
               for (int i = 0; i < 16; ++i) {
                 const float2 x = __ffma2_rn(make_float2(f[c * 32 + 2 * i], f[c * 32 + 2 * i + 1]), sl2v, nbase);
-                const float2 pv = ((FWD_EMU_PAIRS >> (i & 7)) & 1) ? exp2_fma2(x) : make_float2(ex2(x.x), ex2(x.y));
+                const float2 pv = make_float2(ex2(x.x), ex2(x.y));
                 rs2[i & 3] = __fadd2_rn(rs2[i & 3], pv);
                 pk[i] = pack_bf16x2(pv.x, pv.y);
               }

@@ -21,7 +21,9 @@
  * Conventions common to every entry point
  *   - All tensor pointers are DEVICE pointers to contiguous row-major arrays, at least
  *     16-byte aligned.  The caller owns every buffer, workspaces included; the library
- *     never allocates device memory and keeps no state between calls.
+ *     never allocates device memory.  Its only state between calls is the process-wide
+ *     settings of fa_set_wait_limit_ns and fa_set_decode_split and, for
+ *     fa_paged_decode_noalloc, the cached address of its scratch array.
  *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL is the
  *     legacy default stream).  FA_OK means the launch was accepted.  Faults that
  *     happen while the kernel runs surface at the caller's next synchronisation.
@@ -106,8 +108,9 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
 
 /*
  * fa_paged_decode_workspace_size — bytes of device workspace fa_paged_decode needs
- * for the split-KV partial results (fp32 O and lse per split) and per-(request,
- * key/value head) completion counters.  Returns 0 for invalid sizes.
+ * for the split-KV partial results: fp32 O [R,Hq,splits,d] and lse [R,Hq,splits], each
+ * 256-byte aligned, with splits = ceil(max_blocks_per_seq / split size) for the split
+ * size in force (see fa_set_decode_split).  Returns 0 for invalid sizes.
  */
 size_t fa_paged_decode_workspace_size(int R, int Hq, int d, int max_blocks_per_seq, int block_size);
 
@@ -126,6 +129,13 @@ size_t fa_paged_decode_workspace_size(int R, int Hq, int d, int max_blocks_per_s
  *   A physical block id outside [0, num_blocks) or a ctx_len out of range is not
  *   dereferenced: the kernel skips it and sets the device status word
  *   (FA_ERR_INVALID_ARG), so the result for that request is undefined.
+ *   Work split: each request's blocks are cut into splits of a fixed number of blocks
+ *   (fa_set_decode_split), one CTA per (split, key/value head, request); splits of one
+ *   request are merged by their lse weights.  The result does not depend on the split
+ *   size beyond fp32 rounding order.
+ *   If a bounded in-kernel wait runs out (fa_device_status then reports
+ *   FA_ERR_DEVICE_TIMEOUT), o and lse of the affected requests are undefined (the
+ *   kernels write NaN there rather than leftover partial results).
  * Errors: FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_WORKSPACE.
  */
 fa_status fa_paged_decode(const void* q, const void* k_cache, const void* v_cache,
@@ -133,6 +143,16 @@ fa_status fa_paged_decode(const void* q, const void* k_cache, const void* v_cach
                           int R, int Hq, int Hkv, int d, int block_size, int max_blocks_per_seq,
                           int num_blocks, float scale, fa_dtype dtype,
                           void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * fa_set_decode_split — number of cache blocks per split of fa_paged_decode (a multiple
+ * of 4 in [32, 128]; 0 restores the library's default, 128 blocks = 2048 tokens at
+ * block_size 16) for calls made after it, process-wide.  Smaller splits spread long
+ * contexts over more CTAs at the cost of more partial results to merge.  The workspace
+ * size depends on it: query fa_paged_decode_workspace_size after setting it.  Returns
+ * the previous setting, or -1 (and changes nothing) for a value out of range.
+ */
+int fa_set_decode_split(int blocks);
 
 /*
  * fa_paged_prefill — forward pass of a batch of variable-length sequences whose keys and
@@ -201,7 +221,10 @@ fa_status fa_paged_kv_append(const void* k_new, const void* v_new, void* k_cache
  * function never calls cudaMalloc, cudaFree or any allocating library routine.
  *
  * The first call on a device (with that device current) looks up the scratch array's
- * device address and caches it; make that first call before any stream capture.  Every
+ * device address and caches it; make that first call before any stream capture.  The
+ * cache is per CUDA context: after the device's context is destroyed and re-created
+ * (cudaDeviceReset), the next call looks the address up again, so that call too should
+ * come before any capture.  Every
  * call shares the one array, which keeps the last call's contents; nothing in it has to
  * start at zero (each partial the merge reads is written earlier in the same call).
  * Calls that overlap on the GPU (different streams, or different host threads without
@@ -235,14 +258,6 @@ void fa_set_wait_limit_ns(uint64_t ns);
  * timeout path; never faults or hangs the device.
  */
 fa_status fa_selftest_wait_timeout(void* stream);
-
-/*
- * fa_selftest_exp2 — evaluates, for n device floats x (x <= 0), the FMA-pipe 2^x that the
- * forward kernel uses for part of each unmasked score tile (range reduction plus a
- * fitted degree-4 polynomial, relative error <= 2.7e-6 for x in [-126, 0]), writing y.
- * For tests of that approximation against exp2.
- */
-fa_status fa_selftest_exp2(const float* x, float* y, int n, void* stream);
 
 #ifdef __cplusplus
 }

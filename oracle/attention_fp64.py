@@ -15,7 +15,7 @@ Sources (three web pages, cited by title and section):
   [KR] "Kernels de atención rápida y fusión de operadores" (the-ai.news),
        "Atención tipo FlashAttention y atención paginada".
 
-Readings where the pages are silent (each also listed in the design notes):
+Readings where the pages are silent (the plainest reading the rest of the pages supports):
   * LSE is ``m + ln(l)`` over the *scaled* scores, natural log.
   * GQA maps query head h to key/value head ``h // (Hq // Hkv)`` (contiguous groups).
   * Causal masking is bottom-right aligned: query i sits at key position

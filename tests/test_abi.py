@@ -48,6 +48,23 @@ def test_workspace_sizes(L):
     assert L.fa_paged_decode_workspace_size(64, 12, 128, 0, 16) == 0
 
 
+def test_decode_split_setting_sizes_the_workspace(L):
+    """Splits of 32 blocks need four times the partial results of 128-block splits; values
+    outside [32, 128] or not a multiple of 4 are refused and change nothing."""
+    old = L.fa_set_decode_split(128)
+    try:
+        big = L.fa_paged_decode_workspace_size(64, 12, 128, 512, 16)
+        assert L.fa_set_decode_split(32) == 128
+        small = L.fa_paged_decode_workspace_size(64, 12, 128, 512, 16)
+        assert small >= 4 * (big - 512) and small == 64 * 12 * 16 * 128 * 4 + 64 * 12 * 16 * 4
+        for bad in (31, 16, 130, 256, -4, 34):
+            assert L.fa_set_decode_split(bad) == -1
+        assert L.fa_set_decode_split(0) == 32
+        assert L.fa_paged_decode_workspace_size(64, 12, 128, 512, 16) == big
+    finally:
+        L.fa_set_decode_split(old)
+
+
 FAKE = 1 << 20  # 16-byte aligned, never dereferenced: every call below is rejected on the host
 
 

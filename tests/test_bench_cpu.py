@@ -73,3 +73,23 @@ def test_traffic_hash_ignores_comments_only(tmp_path, monkeypatch):
     assert bench.kernel_sources_sha(["k.cuh"]) == h0
     f.write_text("int a = 2;\nint b;\n")
     assert bench.kernel_sources_sha(["k.cuh"]) != h0
+
+
+def test_oracle_row_units_count_the_workload_flops():
+    """One pass over every row unit of a small causal GQA workload (ragged last unit) counts
+    exactly the workload's algorithmic FLOPs, and the units cover every query row once."""
+    c = W.DenseCase("units", 2, 4, 2, 300, 300, 64, "bf16", True, 5)
+    orc = bench.OracleRows(c, rows=128)
+    assert orc.per_head == 3 and orc.units == 2 * 4 * 3
+    for _ in range(orc.units):
+        orc.step()
+    assert orc.rows_done == 2 * 4 * 300
+    assert orc.flops == pytest.approx(c.fwd_flops(), rel=1e-12)
+
+
+def test_compact_secondary_record():
+    r = {"tflops": 1157.123, "per_step_ms": 3.80123,
+         "roofline": {"frac": 0.7031, "traffic": 640e6, "algorithmic_bytes_per_launch": 540e6}}
+    assert bench.compact(r, "tflops") == [1157.12, "TFLOP/s", 3.8012, 0.7031, 1.19]
+    r2 = {"gbs": 5334.04, "per_step_ms": 0.05411, "roofline": {"frac": 0.8138}}
+    assert bench.compact(r2, "gbs", 1) == [5334.0, "GB/s", 0.0541, 0.8138, None]

@@ -63,10 +63,23 @@ def test_bwd_edge_shapes(B, Hq, Hkv, Nq, Nkv, d, causal):
 
 
 def test_bwd_bf16_gradients():
+    """bf16 gradients are the fp32 gradients rounded once.  The fp32 gradients meet the flat
+    bar against the oracle; dK and dV stored as bf16 equal the round-to-nearest-even cast of
+    the fp32 ones bit for bit (same accumulation order); dQ, whose fp32 accumulator takes
+    reductions from many CTAs in no fixed order, is within one bf16 ulp of that cast.  A
+    bf16-stored value can sit half an ulp (up to 0.031 in [8, 16)) from the exact gradient,
+    so bf16 storage alone meets only the relaxed bar of check_bf16_stored."""
     case = DenseCase("bwd_bf16", 1, 4, 2, 640, 640, 64, "bf16", True, 91)
-    (q, k, v, do), (dq, dk, dv) = run(case, torch.bfloat16)
+    (q, k, v, do), (dq32, dk32, dv32) = run(case, torch.float32)
+    (_, _, _, _), (dq, dk, dv) = run(case, torch.bfloat16)
     assert dq.dtype == dk.dtype == dv.dtype == torch.bfloat16
     rq, rk, rv = ora.attention_bwd(q, k, v, do, case.scale, True)
+    for got, ref, n in ((dq32, rq, "dQ"), (dk32, rk, "dK"), (dv32, rv, "dV")):
+        check_bf16(got, ref, n + " (fp32)")
+    assert torch.equal(dk, dk32.to(torch.bfloat16)) and torch.equal(dv, dv32.to(torch.bfloat16))
+    cast = dq32.to(torch.bfloat16).float()
+    ulp = torch.exp2(torch.floor(torch.log2(cast.abs().clamp_min(2.0 ** -126))) - 7)
+    assert ((dq.float() - cast).abs() <= ulp).all()
     over = 0
     for got, ref, n in ((dq, rq, "dQ"), (dk, rk, "dK"), (dv, rv, "dV")):
         over += check_bf16_stored(got, ref, n)

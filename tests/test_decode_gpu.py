@@ -76,3 +76,25 @@ def test_out_of_range_block_id_is_flagged_not_read():
     O, L = oracle({**inp, "block_table": inp["block_table"][:1], "ctx_lens": inp["ctx_lens"][:1],
                    "q": inp["q"][:1]})
     check_bf16(o[:1], O, "untouched request")
+
+
+@pytest.mark.parametrize("split", [32, 64, 128])
+def test_split_size_does_not_change_the_result(split):
+    """The blocks of a request are cut into splits of `split` blocks and the splits' partial
+    results merged by their lse weights ("No basta con promediar los resultados de los
+    bloques"): a different cut of the same keys must give the same attention.  Config 5
+    at each split size against the oracle, and against the default split within the bf16
+    bar (128-block splits: 1-4 per request; 32-block splits: up to 16)."""
+    inp = PAGED_DECODE.make(poison_unused=True)
+    ref_o, ref_lse = run(inp)
+    old = fa.set_decode_split(split)
+    try:
+        o, lse = run(inp)
+    finally:
+        fa.set_decode_split(old)
+    assert fa.device_status() == 0
+    O, L = oracle(inp)
+    check_bf16(o, O, f"O split {split}")
+    check_lse(lse, L, f"lse split {split}")
+    check_bf16(o, ref_o.double().cpu().numpy(), f"O split {split} vs default split")
+    check_lse(lse, ref_lse.double().cpu().numpy(), f"lse split {split} vs default split")

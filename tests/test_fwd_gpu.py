@@ -144,42 +144,50 @@ def test_causal_row0_returns_v0_exactly():
     assert torch.equal(o[:, :, 0].cpu(), vr[:, :, 0])
 
 
-def _sample_rows(n, rng, extra=20):
+def _sample_rows(n, rng, count=512):
+    """Seeded rows of one head: the tile boundaries and ends, plus random rows up to `count`."""
     fixed = [0, 1, 127, 128, 255, 256, 257, n // 2, n - 129, n - 128, n - 2, n - 1]
     rows = set(r for r in fixed if 0 <= r < n)
-    rows.update(int(x) for x in rng.choice(n, size=min(n, extra), replace=False))
+    rest = np.setdiff1d(np.arange(n), np.fromiter(rows, dtype=np.int64))
+    rows.update(int(x) for x in rng.choice(rest, size=min(len(rest), max(0, count - len(rows))), replace=False))
     return sorted(rows)
 
 
-def test_gqa_prefill_causal_full_size():
-    """B=4, Hq=32, Hkv=8, N=8192, d=128, causal: every head on sampled rows, two heads in full."""
-    case = GQA_PREFILL_CAUSAL
-    q, k, v, o, lse = run(case)
-    rng = np.random.default_rng(3)
+def _check_sampled_heads(case, q, k, v, o, lse, rows_per_head=512):
+    """Every (b, h) head on `rows_per_head` seeded rows: O at the bf16 bar (max-abs and
+    relative Frobenius over the sampled block), lse at its bar.  Rows of the forward pass
+    are independent, so the oracle's per-row function is exact for them."""
+    rng = np.random.default_rng(case.seed)
+    qn, kn, vn = ora.to_f64(q), ora.to_f64(k), ora.to_f64(v)
     on, ln = to_np(o), lse.cpu().numpy()
     for b in range(case.B):
         for h in range(case.Hq):
-            rows = _sample_rows(case.Nq, rng, 8)
-            O, L = ora.attention_fwd_rows(q, k, v, case.scale, True, b, h, rows)
-            assert np.abs(on[b, h, rows] - O).max() <= 2e-2
-            assert np.abs(ln[b, h, rows] - L).max() <= 1e-3
-    for b, h in ((0, 0), (3, 31)):
+            rows = _sample_rows(case.Nq, rng, rows_per_head)
+            O, L = ora.attention_fwd_rows(qn, kn, vn, case.scale, case.causal, b, h, rows)
+            check_bf16(on[b, h, rows], O, f"{case.name} O[{b},{h}]")
+            check_lse(ln[b, h, rows], L, f"{case.name} lse[{b},{h}]")
+    return qn, kn, vn, on, ln
+
+
+def test_gqa_prefill_causal_full_size():
+    """B=4, Hq=32, Hkv=8, N=8192, d=128, causal: every head on 512 seeded rows, four heads in full."""
+    case = GQA_PREFILL_CAUSAL
+    q, k, v, o, lse = run(case)
+    qn, kn, vn, on, ln = _check_sampled_heads(case, q, k, v, o, lse)
+    for b, h in ((0, 0), (1, 17), (2, 6), (3, 31)):
         for r0 in range(0, case.Nq, 2048):
             rows = list(range(r0, r0 + 2048))
-            O, L = ora.attention_fwd_rows(q, k, v, case.scale, True, b, h, rows)
-            check_bf16(o[b, h, r0 : r0 + 2048], O, f"O[{b},{h}]")
-            check_lse(lse[b, h, r0 : r0 + 2048], L, "lse")
+            O, L = ora.attention_fwd_rows(qn, kn, vn, case.scale, True, b, h, rows)
+            check_bf16(on[b, h, r0 : r0 + 2048], O, f"O[{b},{h}]")
+            check_lse(ln[b, h, r0 : r0 + 2048], L, "lse")
 
 
 @pytest.mark.parametrize("case", prefill_sweep(), ids=lambda c: c.name)
 def test_noncausal_sweep_sampled(case):
+    """Non-causal sweep at B*N = 32768: every head on 512 seeded rows (N = 1024 and 2048:
+    half or a quarter of all rows)."""
     q, k, v, o, lse = run(case)
-    rng = np.random.default_rng(case.seed)
-    for b, h in ((0, 0), (case.B - 1, case.Hq - 1), (case.B // 2, 13)):
-        rows = _sample_rows(case.Nq, rng, 24)
-        O, L = ora.attention_fwd_rows(q, k, v, case.scale, False, b, h, rows)
-        check_bf16(o[b, h, rows], O, f"{case.name} O[{b},{h}]")
-        check_lse(lse[b, h, rows], L, "lse")
+    _check_sampled_heads(case, q, k, v, o, lse)
 
 
 def test_repeat_calls_are_identical():
@@ -201,20 +209,3 @@ def test_wait_timeout_sets_status_without_fault():
     # the context is still usable
     x = torch.ones(4, device="cuda")
     assert x.sum().item() == 4.0
-
-
-def test_fma_pipe_exp2_against_exp2():
-    """The FMA-pipe 2^x used for part of each unmasked tile stays within 3e-6 of exp2."""
-    import ctypes
-
-    x = torch.cat([torch.linspace(-126.0, 0.0, 1 << 20, dtype=torch.float64),
-                   -torch.rand(1 << 20, dtype=torch.float64, generator=torch.Generator().manual_seed(5)) * 30])
-    xf = x.float().cuda()
-    y = torch.empty_like(xf)
-    st = fa.lib().fa_selftest_exp2(ctypes.c_void_p(xf.data_ptr()), ctypes.c_void_p(y.data_ptr()), xf.numel(),
-                                   ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
-    assert st == 0
-    torch.cuda.synchronize()
-    ref = torch.exp2(xf.double().cpu())
-    rel = ((y.double().cpu() - ref).abs() / ref).max().item()
-    assert rel <= 3e-6, rel

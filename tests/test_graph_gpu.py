@@ -1,12 +1,17 @@
 """CUDA-graph capture of a decode step ("Fusión y CUDA Graphs con torch.compile": a graph
 records a sequence of GPU work and replays it with one submission; it needs stable
-addresses and shapes).  The append + decode C-ABI calls are captured once and replayed on
-new inputs written in place; each replay must equal the eager calls."""
+addresses and shapes, and its results are checked with tolerances that suit the dtype).
+The append + decode C-ABI calls are captured once and replayed on new inputs written in
+place; each replay's cache must equal the oracle's append bit for bit, its output and lse
+must match the oracle's decode on that cache, and it must equal the eager calls."""
+import numpy as np
 import pytest
 import torch
 
 import exact_attention_128_b200 as fa
 from exact_attention_128_b200.workloads import PagedCase, randn
+from oracle import attention_fp64 as ora
+from parity import check_bf16, check_lse
 
 pytestmark = pytest.mark.gpu
 
@@ -24,12 +29,18 @@ def test_append_and_decode_replay_in_a_cuda_graph():
     pos = torch.empty(pc.R, device=dev, dtype=torch.int32)
     ctx = torch.empty(pc.R, device=dev, dtype=torch.int32)
     o = torch.empty_like(q)
+    lse = torch.empty(pc.R, pc.Hq, device=dev, dtype=torch.float32)
     ws = torch.empty(fa.paged_decode_workspace_size(pc.R, pc.Hq, pc.d, pc.max_blocks_per_seq, pc.block_size),
                      device=dev, dtype=torch.uint8)
+    L = fa.lib()
 
     def step():
         fa.paged_kv_append(k_new, v_new, kc, vc, table, pos)
-        fa.paged_decode(q, kc, vc, table, ctx, with_lse=False, workspace=ws, out=o)
+        # the C entry point directly, so the graph also writes lse into a fixed buffer
+        st = L.fa_paged_decode(*(fa._ptr(t) for t in (q, kc, vc, table, ctx, o, lse)), pc.R, pc.Hq, pc.Hkv,
+                               pc.d, pc.block_size, pc.max_blocks_per_seq, inp["num_blocks"],
+                               float(pc.scale), fa.FA_DTYPE_BF16, fa._ptr(ws), ws.numel(), fa._stream())
+        assert st == fa.FA_OK
 
     def load(t):
         base = inp["ctx_lens"].to(torch.int32)
@@ -51,13 +62,22 @@ def test_append_and_decode_replay_in_a_cuda_graph():
         step()
     for t in (1, 2, 3):
         load(t)
-        kc_ref, vc_ref = kc.clone(), vc.clone()
+        kc_before, vc_before = kc.clone(), vc.clone()
         g.replay()
         torch.cuda.synchronize()
-        got = o.clone()
-        kc.copy_(kc_ref)
-        vc.copy_(vc_ref)
+        got_o, got_lse = o.clone(), lse.clone()
+        # oracle: the append on the cache as it was before the replay, then the decode step
+        ek, ev = ora.paged_append(ora.to_f64(kc_before), ora.to_f64(vc_before), table.cpu().numpy(),
+                                  pos.cpu().numpy(), ora.to_f64(k_new), ora.to_f64(v_new), pc.block_size)
+        assert np.array_equal(ora.to_f64(kc), ek) and np.array_equal(ora.to_f64(vc), ev), f"replay {t}: cache"
+        O, LSE = ora.paged_decode(ora.to_f64(q), ek, ev, table.cpu().numpy(), ctx.cpu().numpy(), pc.block_size,
+                                  pc.scale)
+        check_bf16(got_o, O, f"replay {t} O")
+        check_lse(got_lse, LSE, f"replay {t} lse")
+        # and the eager calls on the same inputs give the same bits
+        kc.copy_(kc_before)
+        vc.copy_(vc_before)
         step()
         torch.cuda.synchronize()
-        assert torch.equal(got, o), f"replay {t} differs from the eager calls"
+        assert torch.equal(got_o, o) and torch.equal(got_lse, lse), f"replay {t} differs from the eager calls"
     assert fa.device_status() == 0

@@ -12,6 +12,7 @@ import torch
 
 import exact_attention_128_b200 as fa
 from exact_attention_128_b200.workloads import PAGED_DECODE, PagedCase
+from oracle import attention_fp64 as ora
 from parity import check_bf16, check_lse, to_np
 
 pytestmark = pytest.mark.gpu
@@ -52,6 +53,12 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls():
         o, lse = _noalloc(inp)
         check_bf16(o, to_np(ref_o), "noalloc O")
         check_lse(lse, ref_lse.cpu().numpy(), "noalloc lse")
+        # and against the fp64 oracle on the same inputs
+        d = inp["q"].shape[-1]
+        O, L = ora.paged_decode(inp["q"], inp["k_cache"], inp["v_cache"], inp["block_table"], inp["ctx_lens"], 16,
+                                d ** -0.5)
+        check_bf16(o, O, "noalloc O vs oracle")
+        check_lse(lse, L, "noalloc lse vs oracle")
     assert fa.device_status(reset=True) == fa.FA_OK
 
 
