@@ -31,14 +31,30 @@
 //   3. fa_bwd_finalize_kernel: fp32 dQ accumulator -> bf16 dq (only for bf16 gradients;
 //      fp32 gradients accumulate straight into dq).
 //
-// The scale is folded into dS before it is rounded to bf16, so dK and dQ need no
-// further scaling.  TMEM (512 columns): S^T [0,128), dP^T [128,256), dV, dK (D columns
-// each), and dQ: two buffers of D columns when D = 64, or (D = 128) the dP^T columns,
-// which are free once dK has consumed dS^T.
+// The scale is folded into dS before it is rounded to bf16 (the preprocess stores
+// D_i * scale), so dK and dQ need no further scaling.  TMEM (512 columns): S^T [0,128),
+// dP^T [128,256), dV, dK (D columns each), and dQ: at D = 64 one buffer of 64 columns
+// followed by K_j and V_j as bf16 A operands (32 columns each), so that S^T and dP^T are
+// TS MMAs that read only Q and dO from shared memory; at D = 128 dQ takes the dP^T
+// columns, which are free once dK has consumed dS^T, and S^T and dP^T read K_j and V_j
+// from shared memory.
 #pragma once
 #include "common.cuh"
 
 namespace fa {
+
+// Softmax-gradient warpgroups: 2 (both on query half A, then both on half B) or 4 (two
+// per half, the halves concurrently).  Measured on B200, training workload backward: 2:
+// 1.077 ms, 4: 1.240 ms (80 registers per thread at 768 threads, and half B's chain through
+// the MMA warp gets longer).
+// FA_BWD_B_FIRST 1: half B's next S^T / dP^T are issued before the step's dQ MMA; 0: after
+// it (1.088 vs 1.077 ms with two warpgroups).
+#ifndef FA_BWD_WG
+#define FA_BWD_WG 2
+#endif
+#ifndef FA_BWD_B_FIRST
+#define FA_BWD_B_FIRST 0
+#endif
 
 template <int D>
 struct BwdCfg {
@@ -66,16 +82,25 @@ struct BwdCfg {
   // variant relies on the dynamic shared memory starting 1024-byte aligned and checks it.
   static constexpr int SLACK = (D == 128) ? 0 : 1024;
   static constexpr int SMEM = OFF_BAR + 256 + SLACK;
-  static constexpr int THREADS = 512;
+  // softmax-gradient warpgroups: 4 (two per query half, the halves run concurrently) or 2
+  // (both on half A, then both on half B)
+  static constexpr int NWG = FA_BWD_WG;
+  static_assert(NWG == 2 || NWG == 4, "2 or 4 softmax-gradient warpgroups");
+  static constexpr int WG_DRAIN = 4 + 4 * NWG;  // first dQ drain warp
+  static constexpr int THREADS = 32 * (WG_DRAIN + 4);  // producer, MMA, 2 idle, softmax, 4 dQ drain
   static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DV = 256, COL_DK = 256 + D;
-  static constexpr int NQB = (D == 64) ? 2 : 1;  // dQ TMEM buffers
-  __host__ __device__ static constexpr uint32_t col_dq(int buf) { return D == 64 ? uint32_t(384 + 64 * buf) : COL_DP; }
+  // D = 64: K_j and V_j live in TMEM as the A operands of S^T and dP^T (TS MMAs); each
+  // SS MMA of N = 64 would read 6 KB of shared memory for 0.26 MFLOP, the TS form reads 2 KB
+  static constexpr bool KV_TMEM = (D == 64);
+  static constexpr uint32_t COL_KA = 448, COL_VA = 480;  // D = 64 only: 32 columns each
+  static constexpr int NQB = 1;                          // dQ TMEM buffers
+  __host__ __device__ static constexpr uint32_t col_dq(int) { return D == 64 ? 384u : COL_DP; }
 };
 
 struct BwdParams {
   float* dq_acc;          // fp32 [B,Hq,Nq,D] (the caller's dq when gradients are fp32)
   const float* lse2;      // [B*Hq][Nq_pad] lse * log2(e), +inf past Nq
-  const float* dstat;     // [B*Hq][Nq_pad] D_i, 0 past Nq
+  const float* dstat;     // [B*Hq][Nq_pad] D_i * scale, 0 past Nq
   void* dk;
   void* dv;
   int grad_bf16;
@@ -88,6 +113,7 @@ struct BwdParams {
 
 struct BwdBars {
   uint64_t kv_full;
+  uint64_t kv_tmem;  // D = 64: K_j and V_j copied into TMEM (8 softmax-gradient warps arrive)
   uint64_t qdo_full[2];
   uint64_t qdo_empty[2];
   uint64_t sdp_full[2];  // per query half
@@ -113,13 +139,13 @@ __device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, 
 }
 
 // ------------------------------------------------------------------------------ 1
-// D_i = sum_c dO_ic O_ic per query row; lse2 = lse * log2(e); both padded to Nq_pad.
-// 8 threads per row, each covering D/8 consecutive elements.
+// D_i * scale with D_i = sum_c dO_ic O_ic per query row; lse2 = lse * log2(e); both
+// padded to Nq_pad.  8 threads per row, each covering D/8 consecutive elements.
 template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_preprocess_kernel(const __nv_bfloat16* o, const __nv_bfloat16* dO,
                                                                  const float* lse, float* lse2, float* dstat,
                                                                  float* dq_zero, long total_rows_pad, int Nq,
-                                                                 int Nq_pad, long dq_elems) {
+                                                                 int Nq_pad, long dq_elems, float scale) {
   const long gt = long(blockIdx.x) * blockDim.x + threadIdx.x;
   const long row = gt >> 3;  // padded row index
   const int part = int(gt & 7);
@@ -163,7 +189,7 @@ __global__ void __launch_bounds__(256) fa_bwd_preprocess_kernel(const __nv_bfloa
     acc += __shfl_xor_sync(0xffffffffu, acc, 2);
     acc += __shfl_xor_sync(0xffffffffu, acc, 4);
     if (part == 0) {
-      dstat[row] = q < Nq ? acc : 0.f;
+      dstat[row] = q < Nq ? acc * scale : 0.f;
       lse2[row] = q < Nq ? lse[size_t(bh) * Nq + q] * 1.4426950408889634f : INFINITY;
     }
   }
@@ -187,7 +213,7 @@ __global__ void __launch_bounds__(256) fa_bwd_finalize_kernel(const float* acc, 
 
 // ------------------------------------------------------------------------------ 2
 template <int D, bool CAUSAL>
-__global__ void __launch_bounds__(512, 1)
+__global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     fa_bwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                        const __grid_constant__ CUtensorMap tmDQ, const BwdParams p) {
@@ -217,6 +243,7 @@ __global__ void __launch_bounds__(512, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->kv_full, 1);
+    mbar_init(&bars->kv_tmem, 8);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars->qdo_full[s], 1);
       mbar_init(&bars->qdo_empty[s], 1);
@@ -273,65 +300,80 @@ __global__ void __launch_bounds__(512, 1)
     // ---------------------------------------------------------------- MMA issuer
     // Each step is split into query halves A (rows 0-63) and B (64-127): S^T and dP^T of
     // half B run on the tensor core while half A's softmax-gradient is computed, and
-    // half A's dV/dK MMAs run while half B's is.
-    if (lane == 0 && n_steps > 0) {
+    // half A's dV/dK MMAs run while half B's is.  The whole warp runs this role (so the
+    // descriptors stay warp-uniform); the elected lane issues the MMAs and commits.
+    if (n_steps > 0) {
+      const uint32_t leader = elect_one();
       constexpr uint32_t idKK = idesc_bf16_f32(128, 64, 0);             // S^T, dP^T halves: N = 64
       constexpr uint32_t idTS = idesc_bf16_f32(128, D, 1);              // dV, dK: B (dO, Q) MN-major
       constexpr uint32_t idQ = idesc_bf16_f32(128, D, 1) | (1u << 15);  // dQ: A (dS), B (K) MN-major
+      // base descriptors (128-byte swizzle): K-major operands step 32 B per k-step inside a
+      // 64-column block and 16 KB per block; MN-major ones have 128-row (16 KB) blocks
+      const uint64_t dK = sdesc_sw128(sbase + C::OFF_K, 16, 1024), dV = sdesc_sw128(sbase + C::OFF_V, 16, 1024);
+      const uint64_t dQk = sdesc_sw128(sbase + C::OFF_Q, 16, 1024), dOk = sdesc_sw128(sbase + C::OFF_DO, 16, 1024);
+      const uint64_t dQm = sdesc_sw128(sbase + C::OFF_Q, 128 * 128, 1024);
+      const uint64_t dOm = sdesc_sw128(sbase + C::OFF_DO, 128 * 128, 1024);
+      const uint64_t dSm = sdesc_sw128(sbase + C::OFF_DS, 128 * 128, 1024);
+      const uint64_t dKm = sdesc_sw128(sbase + C::OFF_K, 128 * 128, 1024);
       // S^T and dP^T of query half hf of step s (commit sdp_full[hf])
       auto issue_sdp = [&](int s, int hf) {
-        const int st = s & 1;
-        const uint32_t sQ = sbase + C::OFF_Q + st * C::TILE, sO = sbase + C::OFF_DO + st * C::TILE;
-        // rows [64*hf, 64*hf + 64) of Q and dO: 64 rows * 128 B further in each block
+        const uint32_t qo = (s & 1) * C::TILE + hf * 64 * 128;  // rows [64 hf, 64 hf + 64) of Q, dO
+        // K_j, V_j as A from TMEM (D = 64: 8 columns = 16 bf16 per k-step) or shared memory
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint32_t koff = (ks >> 2) * 128 * 128 + (ks & 3) * 32;
-          mma_ss(tmem + C::COL_S + 64 * hf, sdesc_sw128(sbase + C::OFF_K + koff, 16, 1024),
-                 sdesc_sw128(sQ + koff + hf * 64 * 128, 16, 1024), idKK, ks > 0);
+          if constexpr (C::KV_TMEM)
+            mma_ts_p(tmem + C::COL_S + 64 * hf, tmem + C::COL_KA + ks * 8, desc_add(dQk, qo + koff), idKK, ks > 0,
+                     leader);
+          else
+            mma_ss_p(tmem + C::COL_S + 64 * hf, desc_add(dK, koff), desc_add(dQk, qo + koff), idKK, ks > 0, leader);
         }
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint32_t koff = (ks >> 2) * 128 * 128 + (ks & 3) * 32;
-          mma_ss(tmem + C::COL_DP + 64 * hf, sdesc_sw128(sbase + C::OFF_V + koff, 16, 1024),
-                 sdesc_sw128(sO + koff + hf * 64 * 128, 16, 1024), idKK, ks > 0);
+          if constexpr (C::KV_TMEM)
+            mma_ts_p(tmem + C::COL_DP + 64 * hf, tmem + C::COL_VA + ks * 8, desc_add(dOk, qo + koff), idKK, ks > 0,
+                     leader);
+          else
+            mma_ss_p(tmem + C::COL_DP + 64 * hf, desc_add(dV, koff), desc_add(dOk, qo + koff), idKK, ks > 0, leader);
         }
-        mma_commit(&bars->sdp_full[hf]);
+        mma_commit_p(&bars->sdp_full[hf], leader);
       };
       // dV += P^T dO ; dK += dS^T Q for query half hf of step s (K dimension = 64 queries)
       auto issue_dvdk = [&](int s, int hf) {
-        const int st = s & 1;
-        const uint32_t sQ = sbase + C::OFF_Q + st * C::TILE, sO = sbase + C::OFF_DO + st * C::TILE;
+        const uint32_t so = (s & 1) * C::TILE;
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
           const uint32_t acc = (s > 0 || hf > 0 || ks > 0) ? 1u : 0u;
           const uint32_t roff = (hf * 4 + ks) * 2048;  // 16 query rows per k-step
           const uint32_t pcol = 64 * hf + (ks >> 1) * 32 + (ks & 1) * 8;  // packed P / dS of queries 16ks..
-          mma_ts(tmem + C::COL_DV, tmem + C::COL_S + pcol, sdesc_sw128(sO + roff, 128 * 128, 1024), idTS, acc);
-          mma_ts(tmem + C::COL_DK, tmem + C::COL_DP + pcol, sdesc_sw128(sQ + roff, 128 * 128, 1024), idTS, acc);
+          mma_ts_p(tmem + C::COL_DV, tmem + C::COL_S + pcol, desc_add(dOm, so + roff), idTS, acc, leader);
+          mma_ts_p(tmem + C::COL_DK, tmem + C::COL_DP + pcol, desc_add(dQm, so + roff), idTS, acc, leader);
         }
       };
       // dQ_i = dS K_j (M = queries, K dimension = the 128 keys); then release Q_i, dO_i
       auto issue_dq = [&](int s) -> bool {
-        const int qb = (C::NQB == 2) ? (s & 1) : 0;
-        if constexpr (D == 64) {
-          if (s >= 2 && !mbar_wait(&bars->dq_free[qb], ((s >> 1) - 1) & 1, p.wait_ns, abort_flag, 214)) return false;
+        const int qb = 0;
+        if constexpr (C::EARLY) {  // (D = 128 waits for the drain before the step's dP^T)
+          if (s >= 1 && !warp_wait(&bars->dq_free[0], (s - 1) & 1, p.wait_ns, abort_flag, 214)) return false;
         }
-        const uint32_t sds = sbase + C::OFF_DS + (s % C::DS_BUF) * (128 * 128 * 2);
+        const uint32_t dso = (s % C::DS_BUF) * (128 * 128 * 2);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
-          mma_ss(tmem + C::col_dq(qb), sdesc_sw128(sds + ks * 2048, 128 * 128, 1024),
-                 sdesc_sw128(sbase + C::OFF_K + ks * 2048, 128 * 128, 1024), idQ, ks > 0);
-        mma_commit(&bars->dq_full[qb]);
-        mma_commit(&bars->qdo_empty[s & 1]);
+          mma_ss_p(tmem + C::col_dq(qb), desc_add(dSm, dso + ks * 2048), desc_add(dKm, ks * 2048), idQ, ks > 0, leader);
+        mma_commit_p(&bars->dq_full[qb], leader);
+        mma_commit_p(&bars->qdo_empty[s & 1], leader);
         return true;
       };
-      auto wait_qdo = [&](int s) { return mbar_wait(&bars->qdo_full[s & 1], (s >> 1) & 1, p.wait_ns, abort_flag, 211); };
-      auto wait_ds = [&](int s, int hf) { return mbar_wait(&bars->ds_ready[hf], s & 1, p.wait_ns, abort_flag, 213); };
+      auto wait_qdo = [&](int s) { return warp_wait(&bars->qdo_full[s & 1], (s >> 1) & 1, p.wait_ns, abort_flag, 211); };
+      auto wait_ds = [&](int s, int hf) { return warp_wait(&bars->ds_ready[hf], s & 1, p.wait_ns, abort_flag, 213); };
 
-      bool ok = mbar_wait(&bars->kv_full, 0, p.wait_ns, abort_flag, 210);
+      bool ok = C::KV_TMEM ? warp_wait(&bars->kv_tmem, 0, p.wait_ns, abort_flag, 210)
+                           : warp_wait(&bars->kv_full, 0, p.wait_ns, abort_flag, 210);
       if constexpr (C::EARLY) {
         // half A of step s+1 enters the tensor core as soon as half A of step s is
-        // consumed, so the two softmax warpgroups run staggered by half a step
+        // consumed (and half B's as soon as half B's), so the warpgroups of the two halves
+        // run staggered by half a step
         if (ok && (ok = wait_qdo(0))) {
           tc_fence_after();
           issue_sdp(0, 0);
@@ -349,13 +391,19 @@ __global__ void __launch_bounds__(512, 1)
           if (!(ok = wait_ds(s, 1))) break;
           tc_fence_after();
           issue_dvdk(s, 1);
-          if (!(ok = issue_dq(s))) break;
-          if (s + 1 < n_steps) issue_sdp(s + 1, 1);
+          if (FA_BWD_B_FIRST) {
+            // half B's next scores go before this step's dQ, which no softmax warp waits for
+            if (s + 1 < n_steps) issue_sdp(s + 1, 1);
+            if (!(ok = issue_dq(s))) break;
+          } else {
+            if (!(ok = issue_dq(s))) break;
+            if (s + 1 < n_steps) issue_sdp(s + 1, 1);
+          }
         }
       } else {
         for (int s = 0; s < n_steps && ok; ++s) {
           if (!(ok = wait_qdo(s))) break;
-          if (s > 0 && !(ok = mbar_wait(&bars->dq_free[0], (s - 1) & 1, p.wait_ns, abort_flag, 212))) break;
+          if (s > 0 && !(ok = warp_wait(&bars->dq_free[0], (s - 1) & 1, p.wait_ns, abort_flag, 212))) break;
           tc_fence_after();  // (dP^T overwrites the previous dQ: its drain was awaited above)
           issue_sdp(s, 0);
           issue_sdp(s, 1);
@@ -367,46 +415,80 @@ __global__ void __launch_bounds__(512, 1)
           if (!ok || !(ok = issue_dq(s))) break;
         }
       }
-      if (ok) mma_commit(&bars->dkdv_full);
+      if (ok) mma_commit_p(&bars->dkdv_full, leader);
     }
-  } else if (warp >= 4 && warp < 12) {
+  } else if (warp >= 4 && warp < C::WG_DRAIN) {
     // ---------------------------------------------------------------- softmax-gradient
-    // Both warpgroups work on query half A, then both on half B: warps 4-7 take columns
-    // [0, 32) of the half and warps 8-11 columns [32, 64), so every half has two warps per
-    // SMSP to hide each other's latency.  One thread per key (TMEM lane).
+    // One thread per key (TMEM lane).  With four warpgroups, warps 4-7 and 8-11 take
+    // columns [0, 32) and [32, 64) of query half A and warps 12-15 and 16-19 the same of
+    // half B, so the two halves run at the same time on different warps and one half's
+    // TMEM loads, stores and barriers overlap the other half's exponentials; with two,
+    // warps 4-7 and 8-11 take those columns of half A and then of half B.  Each warp works
+    // in two sub-chunks of 16 columns.
     const int wg = (warp - 4) >> 2;
+    const int wc = wg & 1;                        // 32-column chunk of the half
+    const int hf0 = C::NWG == 4 ? (wg >> 1) : 0;  // first (or only) query half of this warp
     const int wq = warp & 3;
     const int r = wq * 32 + lane;  // key within the tile == TMEM lane
     const int key = k0 + r;
     const uint32_t lane_off = uint32_t(wq * 32) << 16;
     const float sl2 = p.scale_log2, scale = p.scale;
     bool ok = true;
+    if constexpr (C::KV_TMEM) {
+      // key row r of K_j (warps 4-7) or V_j (warps 8-11) from shared memory (128-byte
+      // swizzle: 16-byte chunk u of row r sits at chunk u ^ (r % 8)) into TMEM lane r as 32
+      // columns of bf16 pairs, the A-operand layout of the TS MMAs
+      if (n_steps > 0 && wg < 2) {
+        ok = warp_wait(&bars->kv_full, 0, p.wait_ns, abort_flag, 223);
+        if (ok) {
+          const uint8_t* row = smem + (wg == 0 ? C::OFF_K : C::OFF_V) + r * 128;
+          uint32_t a[32];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const uint4 x = *reinterpret_cast<const uint4*>(row + ((u ^ (r & 7)) << 4));
+            a[4 * u] = x.x;
+            a[4 * u + 1] = x.y;
+            a[4 * u + 2] = x.z;
+            a[4 * u + 3] = x.w;
+          }
+          tmem_st32(tmem + lane_off + (wg == 0 ? C::COL_KA : C::COL_VA), a);
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars->kv_tmem);
+        }
+      }
+    }
     for (int s = 0; s < n_steps && ok; ++s) {
       const int st = s & 1;
       const int i = i_begin + s % n_i;
       ok = warp_wait(&bars->qdo_full[st], (s >> 1) & 1, p.wait_ns, abort_flag, 221);
 #pragma unroll 1
-      for (int hf = 0; hf < 2 && ok; ++hf) {
-        ok = warp_wait(&bars->sdp_full[hf], s & 1, p.wait_ns, abort_flag, 220);
-        if (!ok) break;
-        tc_fence_after();
-        const int q0 = 64 * hf + 32 * wg;  // first query (column) of this thread's chunk
-        // columns q < lim of the chunk are masked for this key; a key past Nkv masks all
-        int lim = 0;
-        if (key >= p.Nkv) lim = 32;
-        else if (CAUSAL) lim = min(32, max(0, key - off - i * C::BM - q0));
-        const float* lse_s = reinterpret_cast<const float*>(smem + C::OFF_STAT + st * 1024) + q0;
-        const float* d_s = lse_s + 128;
-        const bool any_masked = __any_sync(0xffffffffu, lim > 0);
-        uint32_t sv[32], dv[32];
-        tmem_ld32(tmem + lane_off + C::COL_S + q0, sv);
-        tmem_ld32(tmem + lane_off + C::COL_DP + q0, dv);
-        tmem_wait_ld();
-        uint32_t pp[16], pd[16];
+      for (int hf = hf0; hf < (C::NWG == 4 ? hf0 + 1 : 2) && ok; ++hf) {
+      ok = warp_wait(&bars->sdp_full[hf], s & 1, p.wait_ns, abort_flag, 220);
+      if (!ok) break;
+      tc_fence_after();
+      const int q0 = 64 * hf + 32 * wc;  // first query (column) of this warp's chunk
+      // columns q < lim of the chunk are masked for this key; a key past Nkv masks all
+      int lim = 0;
+      if (key >= p.Nkv) lim = 32;
+      else if (CAUSAL) lim = min(32, max(0, key - off - i * C::BM - q0));
+      const float* lse_s = reinterpret_cast<const float*>(smem + C::OFF_STAT + st * 1024) + q0;
+      const float* d_s = lse_s + 128;
+      const bool any_masked = __any_sync(0xffffffffu, lim > 0);
+      // dS (query-major, 128-byte swizzle): half hf is block hf, this chunk units 4wc..4wc+3
+      uint8_t* dsrow = smem + C::OFF_DS + (s % C::DS_BUF) * (128 * 128 * 2) + hf * (128 * 128) + r * 128;
 #pragma unroll
-        for (int e = 0; e < 32; e += 4) {
-          const float4 l4 = *reinterpret_cast<const float4*>(lse_s + e);
-          const float4 d4 = *reinterpret_cast<const float4*>(d_s + e);
+      for (int c = 0; c < 2; ++c) {
+        uint32_t sv[16], dv[16];
+        tmem_ld16(tmem + lane_off + C::COL_S + q0 + 16 * c, sv);
+        tmem_ld16(tmem + lane_off + C::COL_DP + q0 + 16 * c, dv);
+        tmem_wait_ld();
+        uint32_t pp[8], pd[8];
+#pragma unroll
+        for (int e = 0; e < 16; e += 4) {
+          const float4 l4 = *reinterpret_cast<const float4*>(lse_s + 16 * c + e);
+          const float4 d4 = *reinterpret_cast<const float4*>(d_s + 16 * c + e);
           const float2 x01 = __ffma2_rn(make_float2(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])),
                                         make_float2(sl2, sl2), make_float2(-l4.x, -l4.y));
           const float2 x23 = __ffma2_rn(make_float2(__uint_as_float(sv[e + 2]), __uint_as_float(sv[e + 3])),
@@ -414,55 +496,57 @@ __global__ void __launch_bounds__(512, 1)
           float2 p01 = make_float2(ex2(x01.x), ex2(x01.y));
           float2 p23 = make_float2(ex2(x23.x), ex2(x23.y));
           if (any_masked) {
-            if (e < lim) p01.x = 0.f;
-            if (e + 1 < lim) p01.y = 0.f;
-            if (e + 2 < lim) p23.x = 0.f;
-            if (e + 3 < lim) p23.y = 0.f;
+            const int col = 16 * c + e;
+            if (col < lim) p01.x = 0.f;
+            if (col + 1 < lim) p01.y = 0.f;
+            if (col + 2 < lim) p23.x = 0.f;
+            if (col + 3 < lim) p23.y = 0.f;
           }
-          // dS * scale = P * (dP - D) * scale
+          // dS * scale = P * (dP * scale - D * scale)  (d4 holds D * scale)
           const float2 g01 = __fmul2_rn(
-              __fmul2_rn(p01, __fadd2_rn(make_float2(__uint_as_float(dv[e]), __uint_as_float(dv[e + 1])),
-                                         make_float2(-d4.x, -d4.y))),
-              make_float2(scale, scale));
+              p01, __ffma2_rn(make_float2(__uint_as_float(dv[e]), __uint_as_float(dv[e + 1])),
+                              make_float2(scale, scale), make_float2(-d4.x, -d4.y)));
           const float2 g23 = __fmul2_rn(
-              __fmul2_rn(p23, __fadd2_rn(make_float2(__uint_as_float(dv[e + 2]), __uint_as_float(dv[e + 3])),
-                                         make_float2(-d4.z, -d4.w))),
-              make_float2(scale, scale));
+              p23, __ffma2_rn(make_float2(__uint_as_float(dv[e + 2]), __uint_as_float(dv[e + 3])),
+                              make_float2(scale, scale), make_float2(-d4.z, -d4.w)));
           pp[e / 2] = pack_bf16x2(p01.x, p01.y);
           pp[e / 2 + 1] = pack_bf16x2(p23.x, p23.y);
           pd[e / 2] = pack_bf16x2(g01.x, g01.y);
           pd[e / 2 + 1] = pack_bf16x2(g23.x, g23.y);
         }
-        // P^T and dS^T as bf16 pairs over the first 16 of this chunk's own 32 S^T / dP^T
-        // columns (never over columns the other warpgroup is still reading); the dV/dK
-        // MMAs read k-steps 0-1 of the half from chunk 0 and k-steps 2-3 from chunk 1
-        tmem_st16(tmem + lane_off + C::COL_S + q0, pp);
-        tmem_st16(tmem + lane_off + C::COL_DP + q0, pd);
-        // dS (query-major, 128-byte swizzle): half hf is block hf, this chunk units 4wg..4wg+3
-        uint8_t* dsrow = smem + C::OFF_DS + (s % C::DS_BUF) * (128 * 128 * 2) + hf * (128 * 128) + r * 128;
+        // P^T and dS^T as bf16 pairs over the first 8 of the sub-chunk's pair of 8-column
+        // groups: queries 16k..16k+15 of the half land at columns 64hf + (k>>1)*32 + (k&1)*8,
+        // where the dV/dK MMAs read k-step k (columns of S^T / dP^T already consumed)
+        tmem_st8(tmem + lane_off + C::COL_S + q0 + 8 * c, pp);
+        tmem_st8(tmem + lane_off + C::COL_DP + q0 + 8 * c, pd);
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int unit = wg * 4 + u;
+        for (int u = 0; u < 2; ++u) {
+          const int unit = wc * 4 + 2 * c + u;
           *reinterpret_cast<uint4*>(dsrow + ((unit ^ (r & 7)) * 16)) =
               make_uint4(pd[4 * u], pd[4 * u + 1], pd[4 * u + 2], pd[4 * u + 3]);
         }
-        tmem_wait_st();
-        fence_proxy_async_smem();  // dS written by the generic proxy, read by the tensor core
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->ds_ready[hf]);
+      }
+      tmem_wait_st();
+      fence_proxy_async_smem();  // dS written by the generic proxy, read by the tensor core
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->ds_ready[hf]);
       }
     }
-    const int hf = wg;  // epilogue: warps 4-7 write dK, warps 8-11 dV
-    // ---- dK_j (half A warps) and dV_j (half B warps); scale already folded into dS
-    const uint32_t col = hf == 0 ? C::COL_DK : C::COL_DV;
-    void* dst = hf == 0 ? p.dk : p.dv;
+    // ---- dK_j (even warpgroups) and dV_j (odd); with four warpgroups half A's take the
+    // first half of the 32-column chunks and half B's the rest; scale already folded into dS
+    const int hf = hf0;
+    const bool is_dk = wc == 0;
+    const uint32_t col = is_dk ? C::COL_DK : C::COL_DV;
+    void* dst = is_dk ? p.dk : p.dv;
     const size_t base = (size_t(bk) * p.Nkv + key) * p.dout;
+    const int nch = p.dout / 32;
+    const int c_lo = (C::NWG == 2 || hf == 0) ? 0 : (nch + 1) / 2, c_hi = (C::NWG == 4 && hf == 0) ? (nch + 1) / 2 : nch;
     if (ok && n_steps > 0) ok = warp_wait(&bars->dkdv_full, 0, p.wait_ns, abort_flag, 222);
     if (ok && n_steps > 0) {
       tc_fence_after();
 #pragma unroll 1
-      for (int c = 0; c < p.dout / 32; ++c) {
+      for (int c = c_lo; c < c_hi; ++c) {
         uint32_t v[32];
         tmem_ld32(tmem + lane_off + col + c * 32, v);
         tmem_wait_ld();
@@ -486,41 +570,40 @@ __global__ void __launch_bounds__(512, 1)
       }
     } else if (n_steps == 0 && key < p.Nkv) {
       // no query row can see these keys: their gradients are zero
-      for (int c = 0; c < p.dout; c += 4) {
+      for (int c = c_lo * 32; c < c_hi * 32; c += 4) {
         if (p.grad_bf16)
           *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(dst) + base + c) = make_uint2(0, 0);
         else
           *reinterpret_cast<float4*>(static_cast<float*>(dst) + base + c) = make_float4(0, 0, 0, 0);
       }
     }
-  } else if (warp >= 12) {
+  } else if (warp >= C::WG_DRAIN) {
     // ---------------------------------------------------------------- dQ drain (query rows)
     const int wq = warp & 3;
     const int r = wq * 32 + lane;
     const uint32_t lane_off = uint32_t(wq * 32) << 16;
     bool ok = true;
     for (int s = 0; s < n_steps && ok; ++s) {
-      const int qb = (C::NQB == 2) ? (s & 1) : 0;
-      const uint32_t ph = (C::NQB == 2) ? ((s >> 1) & 1) : (s & 1);
-      ok = warp_wait(&bars->dq_full[qb], ph, p.wait_ns, abort_flag, 230);
+      const int qb = 0;
+      ok = warp_wait(&bars->dq_full[qb], s & 1, p.wait_ns, abort_flag, 230);
       if (!ok) break;
       tc_fence_after();
       const int h = hk * G + s / n_i, i = i_begin + s % n_i;
       const int q = i * C::BM + r;
       if constexpr (C::DQ_TMA) {
         uint8_t* stg = smem + C::OFF_DQS + wq * (32 * 64 * 4);  // two 32x32 fp32 boxes
-        uint32_t v[64];
-        tmem_ld32(tmem + lane_off + C::col_dq(qb), *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-        tmem_ld32(tmem + lane_off + C::col_dq(qb) + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
-        tmem_wait_ld();
-        if (lane == 0) bulk_wait_read();  // this warp's previous reduce has read the staging
+        if (lane == 0) bulk_wait_read();  // this warp's previous reduces have read the staging
         __syncwarp();
-#pragma unroll
-        for (int hb = 0; hb < 2; ++hb)
+#pragma unroll 1
+        for (int hb = 0; hb < 2; ++hb) {
+          uint32_t v[32];
+          tmem_ld32(tmem + lane_off + C::col_dq(qb) + 32 * hb, v);
+          tmem_wait_ld();
 #pragma unroll
           for (int u = 0; u < 8; ++u)
             *reinterpret_cast<uint4*>(stg + hb * 4096 + lane * 128 + ((u ^ (lane & 7)) << 4)) =
-                make_uint4(v[32 * hb + 4 * u], v[32 * hb + 4 * u + 1], v[32 * hb + 4 * u + 2], v[32 * hb + 4 * u + 3]);
+                make_uint4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+        }
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {

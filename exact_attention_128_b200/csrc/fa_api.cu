@@ -111,7 +111,9 @@ fa_status launch_fwd_bf16(const CUtensorMap& mq, const CUtensorMap& mk, const CU
   using C = FwdCfg<D, BN>;
   auto kern = fa_fwd_bf16_kernel<D, BN, CAUSAL, PAGED>;
   if (set_smem(kern, C::SMEM) != cudaSuccess) return FA_ERR_CUDA;
-  const long items = long((Nq + 2 * C::BM - 1) / (2 * C::BM)) * prm.BH;
+  const long n_qp = (Nq + 2 * C::BM - 1) / (2 * C::BM);
+  // causal dense items run in units of two query-tile pairs (one CTA per unit at most)
+  const long items = (CAUSAL && !PAGED ? (n_qp + 1) / 2 : n_qp) * prm.BH;
   const long slots = long(sm_count()) * C::CTAS_PER_SM;
   if (slots <= 0) return FA_ERR_CUDA;
   kern<<<int(items < slots ? items : slots), C::THREADS, C::SMEM, st>>>(mq, mk, mv, mo, prm);
@@ -165,15 +167,15 @@ fa_status bwd_launch(const void* q, const void* k, const void* v, const void* o,
   if (d == 64)
     fa_bwd_preprocess_kernel<64><<<pre_blocks, 256, 0, st>>>(
         static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, lse2, dstat, dq_acc,
-        long(rows_pad), Nq, Nq_pad, long(rows) * d);
+        long(rows_pad), Nq, Nq_pad, long(rows) * d, scale);
   else if (d == 96)
     fa_bwd_preprocess_kernel<96><<<pre_blocks, 256, 0, st>>>(
         static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, lse2, dstat, dq_acc,
-        long(rows_pad), Nq, Nq_pad, long(rows) * d);
+        long(rows_pad), Nq, Nq_pad, long(rows) * d, scale);
   else
     fa_bwd_preprocess_kernel<128><<<pre_blocks, 256, 0, st>>>(
         static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, lse2, dstat, dq_acc,
-        long(rows_pad), Nq, Nq_pad, long(rows) * d);
+        long(rows_pad), Nq, Nq_pad, long(rows) * d, scale);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
 
   CUtensorMap mq, mk, mv, mo, mdq;

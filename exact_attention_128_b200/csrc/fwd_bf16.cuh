@@ -10,12 +10,13 @@
 //
 // Persistent kernel: CTAs walk work items (two 128-row query tiles Q0, Q1 of one (batch,
 // query head)), item = blockIdx.x + k * gridDim.x, ordered head-major (non-causal: K/V
-// reuse in L2) or longest-first (causal).  Each item streams the 128-key tiles of its key/value head (GQA: head
+// reuse in L2); causal items go in head-major units of a long and a short item of equal
+// total length (paged causal: longest-first).  Each item streams the 128-key tiles of its key/value head (GQA: head
 // h reads h / (Hq/Hkv)).  The K/V ring and the Q buffers run ahead across item
 // boundaries, so loads for the next item overlap the current item's tail and epilogue.
 //   warp 0      TMA producer: Q0/Q1 per item (QBUF buffers), K_j and V_j into a ring.
-//   warp 1      MMA issuer (one thread): S_t = Q_t K_j^T into TMEM (SS MMA), then
-//               u_t += P_t V_j with P_t read from TMEM (TS MMA).
+//   warp 1      MMA issuer (the warp runs the role, one elected lane issues): S_t = Q_t K_j^T
+//               into TMEM (SS MMA), then u_t += P_t V_j with P_t read from TMEM (TS MMA).
 //   warps 4-7   softmax for Q0, warps 8-11 softmax for Q1: each thread owns one
 //               query row = one TMEM lane; it reads S_t, updates (m, l), writes P_t
 //               (bf16) over S_t in TMEM, rescales u_t in TMEM when m rose, and at the
@@ -137,12 +138,19 @@ __global__ void __launch_bounds__(FwdCfg<D, BN>::THREADS, FwdCfg<D, BN>::CTAS_PE
 
   const int warp = warp_id(), lane = lane_id();
   const int n_qp = (p.Nq + 2 * C::BM - 1) / (2 * C::BM);
-  const int n_items = n_qp * p.BH;
-  // item -> (query-tile pair, batch*head).  Non-causal items are head-major, so the CTAs
-  // running at the same time share one or two heads' K/V in L2 (at N = 8192 this cut
-  // DRAM traffic per launch from 4.2 GB to the 0.64 GB of the algorithm); causal items are
-  // longest-first over all heads (last query tiles first), which balances their very
-  // unequal lengths better than any head grouping measured.
+  // Causal dense items come in units of two query-tile pairs of one head, qt and
+  // n_qp - 1 - qt, whose key ranges add up to the same length for every unit; units are
+  // head-major, so the CTAs running at the same time stream the K/V prefix of one or two
+  // key/value heads and share it in L2, and each CTA runs whole units, which balances the
+  // very unequal causal lengths.  Index it = 2 * unit + (0: the longer pair, 1: the
+  // shorter); the middle pair of an odd n_qp has no partner (index 1 is empty).
+  constexpr bool PAIRS = CAUSAL && !PAGED;
+  const int n_units = (n_qp + 1) / 2;
+  const int n_items = PAIRS ? 2 * n_units * p.BH : n_qp * p.BH;
+  // index of this CTA's k-th item (>= n_items once it has none left)
+  auto item_index = [&](int k) {
+    return PAIRS ? 2 * (int(blockIdx.x) + (k >> 1) * int(gridDim.x)) + (k & 1) : int(blockIdx.x) + k * int(gridDim.x);
+  };
   // keys (L) and query rows (ql) of a sequence; paged mode reads them per request and
   // gives out-of-range lengths no work (flagging them in the status word)
   auto seq_len = [&](int bh, int& L, int& ql) {
@@ -163,22 +171,29 @@ __global__ void __launch_bounds__(FwdCfg<D, BN>::THREADS, FwdCfg<D, BN>::CTAS_PE
   // item -> (query-tile pair qt, batch*head bh, its sequence's L and ql, key tiles n; n = 0:
   // nothing to do).  Non-causal items are head-major, so the CTAs running at the same time
   // share one or two heads' K/V in L2 (at N = 8192 this cut DRAM traffic per launch from
-  // 4.2 GB to the 0.64 GB of the algorithm); causal items are longest-first over all heads
-  // (last query tiles first), which balances their very unequal lengths better than any
-  // head grouping measured.  In paged mode the causal order counts tile pairs from each
-  // request's own last one, so the long items of every request come first.
+  // 4.2 GB to the 0.64 GB of the algorithm); causal items are the paired units above.  In
+  // paged mode the causal order is longest-first over all heads, counting tile pairs from
+  // each request's own last one, so the long items of every request come first.
   struct Item {
     int qt, bh, L, ql, n;
   };
   auto item_of = [&](int it) {
     Item x;
-    x.bh = CAUSAL ? it % p.BH : it / n_qp;
-    seq_len(x.bh, x.L, x.ql);
-    if (CAUSAL && PAGED)
-      x.qt = (x.ql + 2 * C::BM - 1) / (2 * C::BM) - 1 - it / p.BH;
-    else
-      x.qt = CAUSAL ? n_qp - 1 - it / p.BH : it % n_qp;
     x.n = 0;
+    if constexpr (PAIRS) {
+      const int u = it >> 1, a = u % n_units;
+      x.bh = u / n_units;
+      seq_len(x.bh, x.L, x.ql);
+      x.qt = (it & 1) ? a : n_qp - 1 - a;
+      if ((it & 1) && x.qt == n_qp - 1 - a) return x;  // the unpaired middle pair
+    } else {
+      x.bh = CAUSAL ? it % p.BH : it / n_qp;
+      seq_len(x.bh, x.L, x.ql);
+      if (CAUSAL && PAGED)
+        x.qt = (x.ql + 2 * C::BM - 1) / (2 * C::BM) - 1 - it / p.BH;
+      else
+        x.qt = CAUSAL ? n_qp - 1 - it / p.BH : it % n_qp;
+    }
     if (x.qt >= 0 && x.qt * 2 * C::BM < x.ql) {
       int kv_end = x.L;
       if (CAUSAL) kv_end = min(x.L, min(x.qt * 2 * C::BM + 2 * C::BM, x.ql) + (x.L - x.ql));
@@ -227,7 +242,7 @@ __global__ void __launch_bounds__(FwdCfg<D, BN>::THREADS, FwdCfg<D, BN>::CTAS_PE
       int kv = 0;  // K/V tiles issued so far (ring position)
       int local = 0;
       bool ok = true;
-      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+      for (int k = 0, it = item_index(0); it < n_items && ok; it = item_index(++k)) {
         const Item x = item_of(it);
         if (x.n == 0) continue;
         const int zkv = (x.bh / p.Hq) * p.Hkv + (x.bh % p.Hq) / (p.Hq / p.Hkv);
@@ -269,7 +284,7 @@ __global__ void __launch_bounds__(FwdCfg<D, BN>::THREADS, FwdCfg<D, BN>::CTAS_PE
     }
     int kv = 0, local = 0;
     bool ok = true;
-    for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+    for (int k = 0, it = item_index(0); it < n_items && ok; it = item_index(++k)) {
       const Item x = item_of(it);
       if (x.n == 0) continue;
       const int b = x.bh / p.Hq;
@@ -326,53 +341,54 @@ __global__ void __launch_bounds__(FwdCfg<D, BN>::THREADS, FwdCfg<D, BN>::CTAS_PE
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    // The whole warp runs this role so descriptors stay warp-uniform; the elected lane
+    // issues the MMAs and commits.
+    {
+      const uint32_t leader = elect_one();
       constexpr uint32_t idS = idesc_bf16_f32(128, C::BN, 0);  // K-major A (Q) and B (K)
       constexpr uint32_t idPV = idesc_bf16_f32(128, D, 1);     // B (V) is MN-major
+      const uint64_t dQ = sdesc_sw128(sQ, 16, 1024), dK = sdesc_sw128(sK, 16, 1024);
+      const uint64_t dV = sdesc_sw128(sV, C::BN * 128, 1024);
       auto issue_S = [&](int qb, int t, int st) {
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const int kb = ks >> 2, kin = ks & 3;
-          const uint64_t a =
-              sdesc_sw128(sQ + (qb * 2 + t) * C::Q_TILE + kb * C::BM * 128 + kin * 32, 16, 1024);
-          const uint64_t bd = sdesc_sw128(sK + st * C::KV_TILE + kb * C::BN * 128 + kin * 32, 16, 1024);
-          mma_ss(tmem + C::COL_S + t * C::BN, a, bd, idS, ks > 0 ? 1u : 0u);
+          mma_ss_p(tmem + C::COL_S + t * C::BN, desc_add(dQ, (qb * 2 + t) * C::Q_TILE + kb * C::BM * 128 + kin * 32),
+                   desc_add(dK, st * C::KV_TILE + kb * C::BN * 128 + kin * 32), idS, ks > 0 ? 1u : 0u, leader);
         }
       };
       auto issue_PV = [&](int t, int st, int j) {
 #pragma unroll
-        for (int ks = 0; ks < C::BN / 16; ++ks) {
-          const uint64_t bd = sdesc_sw128(sV + st * C::KV_TILE + ks * 16 * 128, C::BN * 128, 1024);
-          mma_ts(tmem + C::COL_O + t * D, tmem + C::COL_S + t * C::BN + ks * 8, bd, idPV,
-                 (j > 0 || ks > 0) ? 1u : 0u);
-        }
+        for (int ks = 0; ks < C::BN / 16; ++ks)
+          mma_ts_p(tmem + C::COL_O + t * D, tmem + C::COL_S + t * C::BN + ks * 8,
+                   desc_add(dV, st * C::KV_TILE + ks * 16 * 128), idPV, (j > 0 || ks > 0) ? 1u : 0u, leader);
       };
       int kv = 0;  // K/V tiles consumed so far (ring position)
       int g = 0;   // query-tile steps so far (s_full / p_full phase)
       int local = 0;
       bool ok = true;
-      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+      for (int k = 0, it = item_index(0); it < n_items && ok; it = item_index(++k)) {
         const Item x = item_of(it);
         const int n = x.n, L = x.L;
         if (n == 0) continue;
         const int qb = local % C::QBUF, quse = local / C::QBUF;
         ++local;
-        ok = mbar_wait(&bars->q_full[qb], quse & 1, p.wait_ns, abort_flag, 20) &&
-             mbar_wait(&bars->k_full[kv % C::NSTAGE], (kv / C::NSTAGE) & 1, p.wait_ns, abort_flag, 21);
+        ok = warp_wait(&bars->q_full[qb], quse & 1, p.wait_ns, abort_flag, 20) &&
+             warp_wait(&bars->k_full[kv % C::NSTAGE], (kv / C::NSTAGE) & 1, p.wait_ns, abort_flag, 21);
         if (!ok) break;
         tc_fence_after();
         issue_S(qb, 0, kv % C::NSTAGE);
-        mma_commit(&bars->s_full[0]);
+        mma_commit_p(&bars->s_full[0], leader);
         issue_S(qb, 1, kv % C::NSTAGE);
-        mma_commit(&bars->s_full[1]);
+        mma_commit_p(&bars->s_full[1], leader);
         // the Q buffer is free once the item's last S has been computed (not its last P.V):
         // the producer then loads the next item's Q while this item's last tile finishes
-        if (n == 1) mma_commit(&bars->q_empty[qb]);
+        if (n == 1) mma_commit_p(&bars->q_empty[qb], leader);
         for (int j = 0; j < n; ++j, ++kv, ++g) {
           const int st = kv % C::NSTAGE;
           const int st2 = (kv + 1) % C::NSTAGE;
           const bool more = j + 1 < n;
-          ok = mbar_wait(&bars->v_full[st], (kv / C::NSTAGE) & 1, p.wait_ns, abort_flag, 22);
+          ok = warp_wait(&bars->v_full[st], (kv / C::NSTAGE) & 1, p.wait_ns, abort_flag, 22);
           if (!ok) break;
           if constexpr (PAGED) {
             // the sequence's last cache block is partly filled: zero the V rows of its
@@ -382,35 +398,36 @@ __global__ void __launch_bounds__(FwdCfg<D, BN>::THREADS, FwdCfg<D, BN>::CTAS_PE
               uint8_t* sv = smem + C::OFF_V + st * C::KV_TILE;
               const int r0 = L - j * C::BN, r1 = (last + 1) * 16 - j * C::BN;
               for (int kb = 0; kb < C::KB; ++kb)
-                for (int i = r0 * 8; i < r1 * 8; ++i)
+                for (int i = r0 * 8 + lane; i < r1 * 8; i += 32)
                   *reinterpret_cast<uint4*>(sv + kb * C::BN * 128 + i * 16) = make_uint4(0, 0, 0, 0);
               fence_proxy_async_smem();
+              __syncwarp();
             }
           }
-          ok = mbar_wait(&bars->p_full[0], g & 1, p.wait_ns, abort_flag, 23);
+          ok = warp_wait(&bars->p_full[0], g & 1, p.wait_ns, abort_flag, 23);
           if (!ok) break;
           tc_fence_after();
           issue_PV(0, st, j);
           if (more) {
-            ok = mbar_wait(&bars->k_full[st2], ((kv + 1) / C::NSTAGE) & 1, p.wait_ns, abort_flag, 24);
+            ok = warp_wait(&bars->k_full[st2], ((kv + 1) / C::NSTAGE) & 1, p.wait_ns, abort_flag, 24);
             if (!ok) break;
             tc_fence_after();
             issue_S(qb, 0, st2);
-            mma_commit(&bars->s_full[0]);
+            mma_commit_p(&bars->s_full[0], leader);
           } else {
-            mma_commit(&bars->o_final[0]);
+            mma_commit_p(&bars->o_final[0], leader);
           }
-          ok = mbar_wait(&bars->p_full[1], g & 1, p.wait_ns, abort_flag, 25);
+          ok = warp_wait(&bars->p_full[1], g & 1, p.wait_ns, abort_flag, 25);
           if (!ok) break;
           tc_fence_after();
           issue_PV(1, st, j);
-          mma_commit(&bars->kv_empty[st]);
+          mma_commit_p(&bars->kv_empty[st], leader);
           if (more) {
             issue_S(qb, 1, st2);
-            mma_commit(&bars->s_full[1]);
-            if (j + 2 == n) mma_commit(&bars->q_empty[qb]);  // that was the item's last S
+            mma_commit_p(&bars->s_full[1], leader);
+            if (j + 2 == n) mma_commit_p(&bars->q_empty[qb], leader);  // that was the item's last S
           } else {
-            mma_commit(&bars->o_final[1]);
+            mma_commit_p(&bars->o_final[1], leader);
           }
         }
       }
@@ -426,7 +443,7 @@ __global__ void __launch_bounds__(FwdCfg<D, BN>::THREADS, FwdCfg<D, BN>::CTAS_PE
     const float sl2 = p.scale_log2;
     int g = 0, local = 0;
     bool ok = true;
-    for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+    for (int k = 0, it = item_index(0); it < n_items && ok; it = item_index(++k)) {
       const Item x = item_of(it);
       const int qt = x.qt, bh = x.bh, L = x.L, ql = x.ql, n = x.n;
       if (n == 0) continue;

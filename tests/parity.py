@@ -12,6 +12,8 @@ LSE_ATOL = 1e-3
 
 
 def to_np(t):
+    if isinstance(t, np.ndarray):
+        return t.astype(np.float64, copy=False)
     return t.detach().float().cpu().numpy().astype(np.float64)
 
 
