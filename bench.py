@@ -766,6 +766,7 @@ def run_secondaries(W, case, dev, world, peaks, no_cpu):
             oracle=None if no_cpu else cpu_oracle_extrapolated(W.TRAIN_CAUSAL, train=True))
     except fa.FAError as e:
         compact_out[W.TRAIN_CAUSAL.name] = detail[W.TRAIN_CAUSAL.name] = {"unavailable": str(e)}
+    put(W.D256_TRAIN.name, measure_train(W.D256_TRAIN, dev, 50, 5, world, peaks), "tflops")
     r = measure_decode(W.PAGED_DECODE, dev, 300, 10, world, peaks)
     put(W.PAGED_DECODE.name, r, "gbs", 1)
     if case.name != W.VIT_BATCHED_BF16.name:
@@ -795,7 +796,7 @@ def main():
     ap.add_argument("--reference-seconds", type=float, default=90.0,
                     help="--impl reference: host-time budget of the whole oracle run")
     ap.add_argument("--only", choices=["prefill_causal", "prefill_noncausal", "train", "decode", "append", "graph",
-                                       "paged_prefill", "d96", "d256", "f32_train", "vit"],
+                                       "paged_prefill", "d96", "d256", "d256_train", "f32_train", "vit"],
                     help="measure just this one secondary workload (for profiling runs) and print it")
     ap.add_argument("--decode-split", type=int, default=0,
                     help="cache blocks per decode split (0: the library's default)")
@@ -831,6 +832,8 @@ def main():
     if args.only:
         if args.only == "train":
             r = measure_train(W.TRAIN_CAUSAL, dev, args.steps, args.warmup, world, peaks)
+        elif args.only == "d256_train":
+            r = measure_train(W.D256_TRAIN, dev, args.steps, args.warmup, world, peaks)
         elif args.only == "decode":
             r = measure_decode(W.PAGED_DECODE, dev, args.steps, args.warmup, world, peaks)
         elif args.only == "append":

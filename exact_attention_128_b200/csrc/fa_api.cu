@@ -11,6 +11,7 @@
 #include "fwd_d256.cuh"
 #include "fwd_f32.cuh"
 #include "bwd_bf16.cuh"
+#include "bwd_d256.cuh"
 #include "bwd_f32.cuh"
 
 #ifndef FA_FWD_D64_BN
@@ -172,11 +173,37 @@ fa_status bwd_launch(const void* q, const void* k, const void* v, const void* o,
     fa_bwd_preprocess_kernel<96><<<pre_blocks, 256, 0, st>>>(
         static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, lse2, dstat, dq_acc,
         long(rows_pad), Nq, Nq_pad, long(rows) * d, scale);
-  else
+  else if (d == 128)
     fa_bwd_preprocess_kernel<128><<<pre_blocks, 256, 0, st>>>(
         static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, lse2, dstat, dq_acc,
         long(rows_pad), Nq, Nq_pad, long(rows) * d, scale);
+  else
+    fa_bwd_preprocess_kernel<256><<<pre_blocks, 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, lse2, dstat, dq_acc,
+        long(rows_pad), Nq, Nq_pad, long(rows) * d, scale);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+
+  if (d == 256) {
+    // one CTA per (128-key tile, batch * kv head, half of the head dimension); 64-row query
+    // steps (bwd_d256.cuh)
+    using C = Bwd256Cfg;
+    CUtensorMap mq, mk, mv, mo;
+    if (!make_map_bf16(&mq, q, d, Nq, B * Hq, C::BM) || !make_map_bf16(&mk, k, d, Nkv, B * Hkv, C::BN) ||
+        !make_map_bf16(&mv, v, d, Nkv, B * Hkv, C::BN) || !make_map_bf16(&mo, dO, d, Nq, B * Hq, C::BM))
+      return FA_ERR_CUDA;
+    BwdParams prm{dq_acc, lse2, dstat, dk, dv, grad_dtype == FA_DTYPE_BF16 ? 1 : 0, d, Hq, Hkv, Nq, Nkv, Nq_pad,
+                  scale, scale * 1.4426950408889634f, g_wait_ns};
+    auto kern = causal ? fa_bwd_d256_kernel<true> : fa_bwd_d256_kernel<false>;
+    if (set_smem(kern, C::SMEM) != cudaSuccess) return FA_ERR_CUDA;
+    kern<<<dim3((Nkv + C::BN - 1) / C::BN, B * Hkv, 2), C::THREADS, C::SMEM, st>>>(mq, mk, mv, mo, prm);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+    if (grad_dtype == FA_DTYPE_BF16) {
+      const long n = long(rows) * d;
+      fa_bwd_finalize_kernel<<<int((n / 4 + 255) / 256), 256, 0, st>>>(dq_ws, static_cast<__nv_bfloat16*>(dq), n);
+      return launched();
+    }
+    return FA_OK;
+  }
 
   CUtensorMap mq, mk, mv, mo, mdq;
   if (!make_map_bf16(&mq, q, d, Nq, B * Hq, 128) || !make_map_bf16(&mk, k, d, Nkv, B * Hkv, 128) ||
@@ -392,7 +419,7 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   }
   if (dtype != FA_DTYPE_BF16) return FA_ERR_UNSUPPORTED;
   if (grad_dtype != FA_DTYPE_F32 && grad_dtype != FA_DTYPE_BF16) return FA_ERR_UNSUPPORTED;
-  if (d != 64 && d != 96 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 96 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
   if (long(B) * Hq > 65535) return FA_ERR_UNSUPPORTED;
   const size_t need = fa_bwd_workspace_size(B, Hq, Nq, d);
   if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return FA_ERR_WORKSPACE;

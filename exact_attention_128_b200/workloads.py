@@ -87,6 +87,9 @@ TRAIN_CAUSAL = DenseCase("train_fwd_bwd_causal_n4096", 8, 16, 16, 4096, 4096, 64
 # Other head dimensions at the prefill sweep's N = 4096 (B*N = 32768 for d = 96).
 D96_PREFILL = DenseCase("d96_prefill_noncausal_n4096", 8, 32, 8, 4096, 4096, 96, "bf16", False, 5)
 D256_PREFILL = DenseCase("d256_prefill_noncausal_n4096", 4, 16, 4, 4096, 4096, 256, "bf16", False, 7)
+# Training step at head dimension 256 (causal, GQA 16/4): the same forward FLOPs as the
+# d = 64 training step, a quarter of its heads.
+D256_TRAIN = DenseCase("d256_train_fwd_bwd_causal_n4096", 2, 16, 4, 4096, 4096, 256, "bf16", True, 8)
 
 
 def prefill_sweep():

@@ -97,8 +97,10 @@ size_t fa_bwd_workspace_size(int B, int Hq, int Nq, int d);
  *   and dv are summed over the Hq/Hkv query heads that share a key/value head.
  *   workspace: at least fa_bwd_workspace_size(B,Hq,Nq,d) bytes, 256-byte aligned;
  *   its contents on entry do not matter.
- *   dtype BF16: d in {64, 96, 128}, tensor-core kernels (d == 96 on the d == 128 kernel).  dtype F32: d == 64 and grad_dtype
- *   F32, CUDA-core kernels (fp32 products throughout).
+ *   dtype BF16: d in {64, 96, 128, 256}, tensor-core kernels (d == 96 on the d == 128
+ *   kernel; d == 256 on a kernel whose CTAs each own one half of the head dimension and
+ *   recompute the full-d score tiles).  dtype F32: d == 64 and grad_dtype F32, CUDA-core
+ *   kernels (fp32 products throughout).
  * Errors: as fa_fwd, plus FA_ERR_WORKSPACE.
  */
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,

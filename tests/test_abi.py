@@ -117,7 +117,9 @@ def bwd_args(**kw):
         (dict(dtype=fa.FA_DTYPE_F32, d=128), fa.FA_ERR_UNSUPPORTED),
         (dict(dtype=fa.FA_DTYPE_F32, grad_dtype=fa.FA_DTYPE_BF16), fa.FA_ERR_UNSUPPORTED),
         (dict(grad_dtype=9), fa.FA_ERR_UNSUPPORTED),
-        (dict(d=256), fa.FA_ERR_UNSUPPORTED),
+        (dict(d=192), fa.FA_ERR_UNSUPPORTED),
+        (dict(d=256, dtype=fa.FA_DTYPE_F32), fa.FA_ERR_UNSUPPORTED),
+        (dict(d=256, ws=None), fa.FA_ERR_WORKSPACE),
         (dict(ws=None), fa.FA_ERR_WORKSPACE),
         (dict(ws_bytes=1000), fa.FA_ERR_WORKSPACE),
         (dict(ws=FAKE + 16), fa.FA_ERR_WORKSPACE),

@@ -8,7 +8,7 @@ import pytest
 import torch
 
 import exact_attention_128_b200 as fa
-from exact_attention_128_b200.workloads import TRAIN_CAUSAL, DenseCase
+from exact_attention_128_b200.workloads import D256_TRAIN, TRAIN_CAUSAL, DenseCase
 from oracle import attention_fp64 as ora
 from parity import check_bf16, check_bf16_stored, to_np
 
@@ -37,6 +37,20 @@ def test_train_causal_full_size_sampled_heads():
         check_bf16(dv[b, h], rv[b, h], f"dV[{b},{h}]")
 
 
+def test_train_d256_causal_sampled_heads():
+    """Head dimension 256 training workload (B=2, Hq=16, Hkv=4, N=4096, causal): the full
+    gradients of two key/value groups (their four query heads each)."""
+    case = D256_TRAIN
+    (q, k, v, do), (dq, dk, dv) = run(case)
+    groups = [(0, 0), (1, 3)]
+    rq, rk, rv = ora.attention_bwd(q, k, v, do, case.scale, True, heads=groups)
+    for b, g in groups:
+        check_bf16(dk[b, g], rk[b, g], f"dK[{b},{g}]")
+        check_bf16(dv[b, g], rv[b, g], f"dV[{b},{g}]")
+        for h in range(4 * g, 4 * g + 4):
+            check_bf16(dq[b, h], rq[b, h], f"dQ[{b},{h}]")
+
+
 EDGE = [
     # B, Hq, Hkv, Nq, Nkv, d, causal
     (1, 1, 1, 1, 1, 64, False),
@@ -49,6 +63,14 @@ EDGE = [
     (1, 2, 1, 513, 513, 128, True),
     (1, 4, 2, 200, 200, 96, True),
     (2, 2, 1, 130, 300, 96, False),
+    # head dimension 256: 64-row query steps, CTAs per half of the head dimension
+    (1, 1, 1, 1, 1, 256, False),
+    (1, 2, 1, 63, 63, 256, True),
+    (1, 2, 2, 65, 65, 256, True),
+    (1, 4, 2, 300, 300, 256, True),
+    (2, 2, 1, 129, 517, 256, False),
+    (1, 3, 1, 100, 612, 256, True),
+    (1, 2, 2, 640, 640, 256, False),
 ]
 
 
@@ -85,6 +107,21 @@ def test_bwd_bf16_gradients():
         over += check_bf16_stored(got, ref, n)
     # the allowance is for a handful of elements next to a rounding midpoint, not a trend
     assert over <= 1e-3 * (dq.numel() + dk.numel() + dv.numel())
+
+
+def test_bwd_d256_bf16_gradients_and_repeat():
+    """Head dimension 256 with bf16 gradients: dK, dV are the round-to-nearest-even cast of
+    the fp32 ones; two calls give the same dK, dV bits (each key tile's accumulation order
+    is fixed)."""
+    case = DenseCase("bwd256_bf16", 1, 4, 1, 384, 384, 256, "bf16", True, 95)
+    (q, k, v, do), (dq32, dk32, dv32) = run(case, torch.float32)
+    (_, _, _, _), (dq, dk, dv) = run(case, torch.bfloat16)
+    rq, rk, rv = ora.attention_bwd(q, k, v, do, case.scale, True)
+    for got, ref, n in ((dq32, rq, "dQ"), (dk32, rk, "dK"), (dv32, rv, "dV")):
+        check_bf16(got, ref, n + " (fp32, d=256)")
+    assert torch.equal(dk, dk32.to(torch.bfloat16)) and torch.equal(dv, dv32.to(torch.bfloat16))
+    (_, _, _, _), (_, dk32b, dv32b) = run(case, torch.float32)
+    assert torch.equal(dk32, dk32b) and torch.equal(dv32, dv32b)
 
 
 def test_bwd_gradient_invariants_on_gpu():

@@ -441,3 +441,19 @@ def test_paged_prefill_equals_dense_and_decode():
     np.testing.assert_allclose(L1[:, :, 0], Ldd, atol=1e-14)
     with pytest.raises(ValueError):
         ora.paged_prefill(q, kc, vc, table, ctx, [2, 10, 3], bs, 0.5, True)
+
+
+def test_single_key_gradients_are_zero_in_the_oracle():
+    """With one key every softmax row is [1], so dS = P (dP - D) = 0 and dQ = dK = 0 up to
+    fp64 rounding (the case the parity checker compares by max-abs only)."""
+    import sys
+    import os
+    sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
+    from parity import _exactly_zero
+
+    rng = np.random.default_rng(3)
+    q, k, v, do = (rng.standard_normal((1, 1, n, 8)) for n in (5, 1, 1, 5))
+    dq, dk, dv = ora.attention_bwd(q, k, v, do, 0.3, False)
+    assert _exactly_zero(dq) and _exactly_zero(dk)
+    assert np.allclose(dv[0, 0, 0], do[0, 0].sum(axis=0))
+    assert not _exactly_zero(dv)
