@@ -43,15 +43,8 @@
 
 namespace fa {
 
-// Softmax-gradient warpgroups: 2 (both on query half A, then both on half B) or 4 (two
-// per half, the halves concurrently).  Measured on B200, training workload backward: 2:
-// 1.077 ms, 4: 1.240 ms (80 registers per thread at 768 threads, and half B's chain through
-// the MMA warp gets longer).
 // FA_BWD_B_FIRST 1: half B's next S^T / dP^T are issued before the step's dQ MMA; 0: after
-// it (1.088 vs 1.077 ms with two warpgroups).
-#ifndef FA_BWD_WG
-#define FA_BWD_WG 2
-#endif
+// it (measured on B200, training workload backward: 1.088 vs 1.077 ms).
 #ifndef FA_BWD_B_FIRST
 #define FA_BWD_B_FIRST 0
 #endif
@@ -82,12 +75,12 @@ struct BwdCfg {
   // variant relies on the dynamic shared memory starting 1024-byte aligned and checks it.
   static constexpr int SLACK = (D == 128) ? 0 : 1024;
   static constexpr int SMEM = OFF_BAR + 256 + SLACK;
-  // softmax-gradient warpgroups: 4 (two per query half, the halves run concurrently) or 2
-  // (both on half A, then both on half B)
-  static constexpr int NWG = FA_BWD_WG;
-  static_assert(NWG == 2 || NWG == 4, "2 or 4 softmax-gradient warpgroups");
-  static constexpr int WG_DRAIN = 4 + 4 * NWG;  // first dQ drain warp
-  static constexpr int THREADS = 32 * (WG_DRAIN + 4);  // producer, MMA, 2 idle, softmax, 4 dQ drain
+  static constexpr int WG_DRAIN = 12;  // first dQ drain warp
+  static constexpr int THREADS = 512;  // producer, MMA, 2 idle, 8 softmax-gradient, 4 dQ drain
+  // epilogue staging (the Q / dO stages, free by then): per softmax warp, its 32 key rows
+  // of dK or dV as D / 32 swizzled boxes of 32 rows x 128 bytes (fp32; bf16 uses half)
+  static constexpr int STG_WARP = (D / 32) * 4096;
+  static_assert(8 * STG_WARP <= 4 * TILE, "epilogue staging must fit the Q and dO stages");
   static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DV = 256, COL_DK = 256 + D;
   // D = 64: K_j and V_j live in TMEM as the A operands of S^T and dP^T (TS MMAs); each
   // SS MMA of N = 64 would read 6 KB of shared memory for 0.26 MFLOP, the TS form reads 2 KB
@@ -216,8 +209,10 @@ template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     fa_bwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
-                       const __grid_constant__ CUtensorMap tmDQ, const BwdParams p) {
-  // tmO maps dO (same geometry as Q); tmDQ maps the fp32 dQ accumulator (32 x 32 boxes)
+                       const __grid_constant__ CUtensorMap tmDQ, const __grid_constant__ CUtensorMap tmDK,
+                       const __grid_constant__ CUtensorMap tmDV, const BwdParams p) {
+  // tmO maps dO (same geometry as Q); tmDQ maps the fp32 dQ accumulator (32 x 32 boxes);
+  // tmDK, tmDV map dk, dv: fp32 with 32 x 32 boxes or bf16 with 64 x 32 boxes (128-byte swizzle)
   using C = BwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   if (C::SLACK == 0 && (smem_u32(smem_raw) & 1023u) != 0) {  // uniform across the CTA
@@ -419,15 +414,11 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     }
   } else if (warp >= 4 && warp < C::WG_DRAIN) {
     // ---------------------------------------------------------------- softmax-gradient
-    // One thread per key (TMEM lane).  With four warpgroups, warps 4-7 and 8-11 take
-    // columns [0, 32) and [32, 64) of query half A and warps 12-15 and 16-19 the same of
-    // half B, so the two halves run at the same time on different warps and one half's
-    // TMEM loads, stores and barriers overlap the other half's exponentials; with two,
-    // warps 4-7 and 8-11 take those columns of half A and then of half B.  Each warp works
-    // in two sub-chunks of 16 columns.
-    const int wg = (warp - 4) >> 2;
-    const int wc = wg & 1;                        // 32-column chunk of the half
-    const int hf0 = C::NWG == 4 ? (wg >> 1) : 0;  // first (or only) query half of this warp
+    // One thread per key (TMEM lane).  Warps 4-7 and 8-11 take columns [0, 32) and
+    // [32, 64) of query half A and then of half B, in two sub-chunks of 16 columns each.
+    // (Four warpgroups, two per half with the halves running concurrently, were measured
+    // slower: 1.240 against 1.077 ms for the training backward, at 80 registers per thread.)
+    const int wc = (warp - 4) >> 2;  // 32-column chunk of each half
     const int wq = warp & 3;
     const int r = wq * 32 + lane;  // key within the tile == TMEM lane
     const int key = k0 + r;
@@ -438,10 +429,10 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       // key row r of K_j (warps 4-7) or V_j (warps 8-11) from shared memory (128-byte
       // swizzle: 16-byte chunk u of row r sits at chunk u ^ (r % 8)) into TMEM lane r as 32
       // columns of bf16 pairs, the A-operand layout of the TS MMAs
-      if (n_steps > 0 && wg < 2) {
+      if (n_steps > 0) {
         ok = warp_wait(&bars->kv_full, 0, p.wait_ns, abort_flag, 223);
         if (ok) {
-          const uint8_t* row = smem + (wg == 0 ? C::OFF_K : C::OFF_V) + r * 128;
+          const uint8_t* row = smem + (wc == 0 ? C::OFF_K : C::OFF_V) + r * 128;
           uint32_t a[32];
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
@@ -451,7 +442,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
             a[4 * u + 2] = x.z;
             a[4 * u + 3] = x.w;
           }
-          tmem_st32(tmem + lane_off + (wg == 0 ? C::COL_KA : C::COL_VA), a);
+          tmem_st32(tmem + lane_off + (wc == 0 ? C::COL_KA : C::COL_VA), a);
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
@@ -464,7 +455,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       const int i = i_begin + s % n_i;
       ok = warp_wait(&bars->qdo_full[st], (s >> 1) & 1, p.wait_ns, abort_flag, 221);
 #pragma unroll 1
-      for (int hf = hf0; hf < (C::NWG == 4 ? hf0 + 1 : 2) && ok; ++hf) {
+      for (int hf = 0; hf < 2 && ok; ++hf) {
       ok = warp_wait(&bars->sdp_full[hf], s & 1, p.wait_ns, abort_flag, 220);
       if (!ok) break;
       tc_fence_after();
@@ -533,44 +524,54 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       if (lane == 0) mbar_arrive(&bars->ds_ready[hf]);
       }
     }
-    // ---- dK_j (even warpgroups) and dV_j (odd); with four warpgroups half A's take the
-    // first half of the 32-column chunks and half B's the rest; scale already folded into dS
-    const int hf = hf0;
+    // ---- dK_j (warps 4-7) and dV_j (warps 8-11); the scale is already folded into dS.
+    // Each warp stages its 32 key rows in shared memory (128-byte swizzle) and writes them
+    // with TMA tensor stores, which drop the rows past Nkv and the columns past dout.
     const bool is_dk = wc == 0;
     const uint32_t col = is_dk ? C::COL_DK : C::COL_DV;
-    void* dst = is_dk ? p.dk : p.dv;
-    const size_t base = (size_t(bk) * p.Nkv + key) * p.dout;
-    const int nch = p.dout / 32;
-    const int c_lo = (C::NWG == 2 || hf == 0) ? 0 : (nch + 1) / 2, c_hi = (C::NWG == 4 && hf == 0) ? (nch + 1) / 2 : nch;
+    const CUtensorMap* tmap = is_dk ? &tmDK : &tmDV;
     if (ok && n_steps > 0) ok = warp_wait(&bars->dkdv_full, 0, p.wait_ns, abort_flag, 222);
     if (ok && n_steps > 0) {
       tc_fence_after();
+      uint8_t* stg = smem + C::OFF_Q + (warp - 4) * C::STG_WARP;  // every MMA is done: Q, dO free
+      const int nch = p.dout / 32;
 #pragma unroll 1
-      for (int c = c_lo; c < c_hi; ++c) {
+      for (int c = 0; c < nch; ++c) {
         uint32_t v[32];
         tmem_ld32(tmem + lane_off + col + c * 32, v);
         tmem_wait_ld();
-        if (key < p.Nkv) {
-          if (p.grad_bf16) {
-            uint4* o4 = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(dst) + base + c * 32);
+        if (p.grad_bf16) {
+          // 64-column boxes of 32 rows x 128 bytes: chunk c fills half c & 1 of box c / 2
+          uint8_t* row = stg + (c >> 1) * 4096 + lane * 128;
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4)
-              o4[q4] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * q4]), __uint_as_float(v[8 * q4 + 1])),
-                                  pack_bf16x2(__uint_as_float(v[8 * q4 + 2]), __uint_as_float(v[8 * q4 + 3])),
-                                  pack_bf16x2(__uint_as_float(v[8 * q4 + 4]), __uint_as_float(v[8 * q4 + 5])),
-                                  pack_bf16x2(__uint_as_float(v[8 * q4 + 6]), __uint_as_float(v[8 * q4 + 7])));
-          } else {
-            float4* o4 = reinterpret_cast<float4*>(static_cast<float*>(dst) + base + c * 32);
+          for (int u = 0; u < 4; ++u)
+            *reinterpret_cast<uint4*>(row + (((4 * (c & 1) + u) ^ (lane & 7)) << 4)) =
+                make_uint4(pack_bf16x2(__uint_as_float(v[8 * u]), __uint_as_float(v[8 * u + 1])),
+                           pack_bf16x2(__uint_as_float(v[8 * u + 2]), __uint_as_float(v[8 * u + 3])),
+                           pack_bf16x2(__uint_as_float(v[8 * u + 4]), __uint_as_float(v[8 * u + 5])),
+                           pack_bf16x2(__uint_as_float(v[8 * u + 6]), __uint_as_float(v[8 * u + 7])));
+        } else {
+          uint8_t* row = stg + c * 4096 + lane * 128;
 #pragma unroll
-            for (int q4 = 0; q4 < 8; ++q4)
-              o4[q4] = make_float4(__uint_as_float(v[4 * q4]), __uint_as_float(v[4 * q4 + 1]),
-                                   __uint_as_float(v[4 * q4 + 2]), __uint_as_float(v[4 * q4 + 3]));
-          }
+          for (int u = 0; u < 8; ++u)
+            *reinterpret_cast<uint4*>(row + ((u ^ (lane & 7)) << 4)) =
+                make_uint4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
         }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        const int nbox = p.grad_bf16 ? (nch + 1) / 2 : nch;
+        for (int x = 0; x < nbox; ++x)
+          tma_store_3d(tmap, stg + x * 4096, x * (p.grad_bf16 ? 64 : 32), k0 + wq * 32, bk);
+        bulk_commit();
+        bulk_wait_all();  // the stores have read the staging before the CTA ends
       }
     } else if (n_steps == 0 && key < p.Nkv) {
       // no query row can see these keys: their gradients are zero
-      for (int c = c_lo * 32; c < c_hi * 32; c += 4) {
+      void* dst = is_dk ? p.dk : p.dv;
+      const size_t base = (size_t(bk) * p.Nkv + key) * p.dout;
+      for (int c = 0; c < p.dout; c += 4) {
         if (p.grad_bf16)
           *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(dst) + base + c) = make_uint2(0, 0);
         else

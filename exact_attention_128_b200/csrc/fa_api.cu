@@ -125,13 +125,13 @@ int round_up(int x, int m) { return (x + m - 1) / m * m; }
 
 template <int D, bool CAUSAL>
 fa_status launch_bwd_kernel(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                            const CUtensorMap& mo, const CUtensorMap& mdq, const BwdParams& prm, int B, int Hkv,
-                            int Nkv, cudaStream_t st) {
+                            const CUtensorMap& mo, const CUtensorMap& mdq, const CUtensorMap& mdk,
+                            const CUtensorMap& mdv, const BwdParams& prm, int B, int Hkv, int Nkv, cudaStream_t st) {
   using C = BwdCfg<D>;
   auto kern = fa_bwd_bf16_kernel<D, CAUSAL>;
   if (set_smem(kern, C::SMEM) != cudaSuccess) return FA_ERR_CUDA;
   dim3 grid((Nkv + C::BN - 1) / C::BN, B * Hkv);
-  kern<<<grid, C::THREADS, C::SMEM, st>>>(mq, mk, mv, mo, mdq, prm);
+  kern<<<grid, C::THREADS, C::SMEM, st>>>(mq, mk, mv, mo, mdq, mdk, mdv, prm);
   return launched();
 }
 
@@ -205,10 +205,14 @@ fa_status bwd_launch(const void* q, const void* k, const void* v, const void* o,
     return FA_OK;
   }
 
-  CUtensorMap mq, mk, mv, mo, mdq;
+  CUtensorMap mq, mk, mv, mo, mdq, mdk, mdv;
   if (!make_map_bf16(&mq, q, d, Nq, B * Hq, 128) || !make_map_bf16(&mk, k, d, Nkv, B * Hkv, 128) ||
       !make_map_bf16(&mv, v, d, Nkv, B * Hkv, 128) || !make_map_bf16(&mo, dO, d, Nq, B * Hq, 128) ||
       !make_map_f32(&mdq, dq_acc, d, Nq, B * Hq))
+    return FA_ERR_CUDA;
+  // dk, dv for the epilogue's TMA stores
+  if (grad_dtype == FA_DTYPE_BF16 ? !make_map_bf16(&mdk, dk, d, Nkv, B * Hkv, 32) || !make_map_bf16(&mdv, dv, d, Nkv, B * Hkv, 32)
+                                  : !make_map_f32(&mdk, dk, d, Nkv, B * Hkv) || !make_map_f32(&mdv, dv, d, Nkv, B * Hkv))
     return FA_ERR_CUDA;
   // d = 96 runs the d = 128 kernel on 96-wide maps (zero-filled columns 96..127); its
   // gradient rows are written 96 wide
@@ -216,11 +220,11 @@ fa_status bwd_launch(const void* q, const void* k, const void* v, const void* o,
                 scale, scale * 1.4426950408889634f, g_wait_ns};
   fa_status s;
   if (d == 64)
-    s = causal ? launch_bwd_kernel<64, true>(mq, mk, mv, mo, mdq, prm, B, Hkv, Nkv, st)
-               : launch_bwd_kernel<64, false>(mq, mk, mv, mo, mdq, prm, B, Hkv, Nkv, st);
+    s = causal ? launch_bwd_kernel<64, true>(mq, mk, mv, mo, mdq, mdk, mdv, prm, B, Hkv, Nkv, st)
+               : launch_bwd_kernel<64, false>(mq, mk, mv, mo, mdq, mdk, mdv, prm, B, Hkv, Nkv, st);
   else
-    s = causal ? launch_bwd_kernel<128, true>(mq, mk, mv, mo, mdq, prm, B, Hkv, Nkv, st)
-               : launch_bwd_kernel<128, false>(mq, mk, mv, mo, mdq, prm, B, Hkv, Nkv, st);
+    s = causal ? launch_bwd_kernel<128, true>(mq, mk, mv, mo, mdq, mdk, mdv, prm, B, Hkv, Nkv, st)
+               : launch_bwd_kernel<128, false>(mq, mk, mv, mo, mdq, mdk, mdv, prm, B, Hkv, Nkv, st);
   if (s != FA_OK) return s;
   if (grad_dtype == FA_DTYPE_BF16) {
     const long n = long(rows) * d;
