@@ -425,10 +425,17 @@ def measure_train(case, dev, steps, warmup, world, peaks):
                              "frac": round(tflops / peak, 4), "peak_kind": "fp32 FFMA, 148 SMs x 128 lanes x 2 x max clock",
                              "algorithmic_flops_per_step": flops}}
     peak = peaks["bf16_tflops"]
+    # the backward dominates the step; its algorithmic bytes: q, k, v, o, dO (bf16) and lse
+    # read, dq, dk, dv (fp32) written
+    n_q, n_kv = case.B * case.Hq * case.Nq * case.d, case.B * case.Hkv * case.Nkv * case.d
+    bwd_bytes = 2 * (2 * n_q + 2 * n_kv + n_q) + 4 * case.B * case.Hq * case.Nq + 4 * (n_q + 2 * n_kv)
+    kname = f"fa_bwd_d256_kernel<{str(case.causal).lower()}>" if case.d == 256 else \
+        f"fa_bwd_bf16_kernel<{64 if case.d == 64 else 128},{str(case.causal).lower()}>"
     return {"per_step_ms": per, "tflops": tflops,
             "roofline": {"bound": "tensor", "achieved": round(tflops, 2), "peak": peak, "unit": "TFLOP/s",
                          "frac": round(tflops / peak, 4), "frac_of_nominal_2250": round(tflops / NOMINAL_BF16_TFLOPS, 4),
-                         "algorithmic_flops_per_step": flops}}
+                         "algorithmic_flops_per_step": flops, "kernel": kname, "traffic": traffic_for(kname),
+                         "algorithmic_bytes_per_launch": bwd_bytes}}
 
 
 def measure_decode(pc, dev, steps, warmup, world, peaks):
@@ -472,8 +479,9 @@ def measure_decode(pc, dev, steps, warmup, world, peaks):
     return {"per_step_ms": per, "gbs": gbs, "kv_bytes": kvb,
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(gbs / peak, 4), "frac_of_nominal_8000": round(gbs / NOMINAL_HBM_GBS, 4),
-                         "algorithmic_bytes_per_step": kvb, "kernels": ["fa_paged_decode_kernel",
-                                                                        "fa_paged_decode_combine_kernel"]}}
+                         "algorithmic_bytes_per_step": kvb, "algorithmic_bytes_per_launch": kvb,
+                         "kernel": "fa_paged_decode_kernel", "traffic": traffic_for("fa_paged_decode_kernel"),
+                         "kernels": ["fa_paged_decode_kernel", "fa_paged_decode_combine_kernel"]}}
 
 
 def measure_paged_prefill(pc, dev, steps, warmup, world, peaks, peak_key="bf16_tflops"):
