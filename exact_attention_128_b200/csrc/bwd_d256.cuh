@@ -12,14 +12,16 @@
 //     both do; 40 % more MMA work than the five contractions of the method),
 //   - accumulates dV[:, h] and dK[:, h] in TMEM,
 //   - computes dQ^T[h] = K[:, h]^T dS^T (M = the 128 columns of h, N = the step's queries)
-//     and adds it into the fp32 dQ accumulator with coalesced reductions.
+//     and adds it, transposed through shared memory, into the fp32 dQ accumulator with
+//     TMA reduce-adds.
 // Query steps are 64 rows; Q and dO are double-buffered.  V lives in TMEM as the A operand
 // of dP^T (copied once from shared memory), which frees the shared memory it would take.
 //
 // TMEM (512 columns): S^T [0, 64), dP^T [64, 128) (dQ^T after dK has consumed dS^T),
 // dV_h [128, 256), dK_h [256, 384), V [384, 512) (bf16 pairs, 128 columns for 256 d).
 // Shared memory: K 64 KB (four [128 keys][64 d] swizzled blocks), dO stages 2 x 32 KB (V
-// is staged there first), Q stages 2 x 32 KB, dS^T [128 keys][64 queries] 16 KB, lse/D.
+// is staged there first), Q stages 2 x 32 KB, dS^T [128 keys][64 queries] 16 KB, lse/D,
+// dQ staging 16 KB.
 // Roles: warp 0 TMA producer, warp 1 MMA issuer (elected lane), warps 4-11 softmax-
 // gradient (one thread per key; warps 4-7 queries [0, 32), warps 8-11 [32, 64)), warps
 // 12-15 dQ^T drain (one thread per d-row of the half).
@@ -39,7 +41,8 @@ struct Bwd256Cfg {
   static constexpr int OFF_Q = OFF_DO + 65536;   // + st * 32768
   static constexpr int OFF_DS = OFF_Q + 65536;   // [128 keys][64 queries] bf16, 128-byte swizzle
   static constexpr int OFF_STAT = OFF_DS + 16384;  // + st * 512: lse2[64], D[64]
-  static constexpr int OFF_BAR = OFF_STAT + 1024;
+  static constexpr int OFF_DQS = OFF_STAT + 1024;   // dQ staging: per drain warp [32 queries][32 d] fp32
+  static constexpr int OFF_BAR = OFF_DQS + 4 * 4096;
   static constexpr int SMEM = OFF_BAR + 256 + 1024;
   static constexpr int THREADS = 512;
   static constexpr uint32_t COL_S = 0, COL_DP = 64, COL_DV = 128, COL_DK = 256, COL_VA = 384;
@@ -63,8 +66,9 @@ template <bool CAUSAL>
 __global__ void __launch_bounds__(Bwd256Cfg::THREADS, 1)
     fa_bwd_d256_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
-                       const BwdParams p) {
-  // tmQ / tmO map Q and dO with (64, 64) boxes, tmK / tmV map K and V with (64, 128) boxes
+                       const __grid_constant__ CUtensorMap tmDQ, const BwdParams p) {
+  // tmQ / tmO map Q and dO with (64, 64) boxes, tmK / tmV map K and V with (64, 128) boxes,
+  // tmDQ the fp32 dQ accumulator with (32, 32) boxes and the 128-byte swizzle
   using C = Bwd256Cfg;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -363,33 +367,44 @@ __global__ void __launch_bounds__(Bwd256Cfg::THREADS, 1)
     }
   } else if (warp >= 12) {
     // ---------------------------------------------------------------- dQ^T drain
-    // Thread r holds d-column h * 128 + r of the step's 64 queries; for each query the warp's
-    // 32 lanes add 32 consecutive floats of that query's dQ row.
+    // Thread r holds d-column h * 128 + r of the step's 64 queries.  The warp reads all 64
+    // columns from TMEM, releases them (the next step's dP^T may overwrite them), then for
+    // each half of the queries writes a transposed [32 queries][32 d] fp32 tile (each query a
+    // 128-byte row, 128-byte swizzle) and adds it into the fp32 accumulator with a TMA
+    // reduce-add.
     const int wq = warp & 3;
-    const int r = wq * 32 + lane;
     const uint32_t lane_off = uint32_t(wq * 32) << 16;
+    uint8_t* stg = smem + C::OFF_DQS + wq * 4096;
     bool ok = true;
     for (int s = 0; s < n_steps && ok; ++s) {
       ok = warp_wait(&bars->dq_full, s & 1, p.wait_ns, abort_flag, 330);
       if (!ok) break;
       tc_fence_after();
       const int h = hk * G + s / n_i, i = i_begin + s % n_i;
-      float* dst = p.dq_acc + (size_t(b) * p.Hq + h) * p.Nq * size_t(C::D) + hh * C::DH + r;
-#pragma unroll 1
-      for (int c = 0; c < 2; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tmem + lane_off + C::COL_DP + 32 * c, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int q = i * C::BM + 32 * c + e;
-          if (q < p.Nq) atomicAdd(dst + size_t(q) * C::D, __uint_as_float(v[e]));
-        }
-      }
+      uint32_t v0[32], v1[32];
+      tmem_ld32(tmem + lane_off + C::COL_DP, v0);
+      tmem_ld32(tmem + lane_off + C::COL_DP + 32, v1);
+      tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->dq_free);
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        if (lane == 0) bulk_wait_read();  // the previous reduce-add has read the staging
+        __syncwarp();
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+          *reinterpret_cast<uint32_t*>(stg + e * 128 + (((lane >> 2) ^ (e & 7)) << 4) + (lane & 3) * 4) =
+              c == 0 ? v0[e] : v1[e];
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_reduce_add_3d(&tmDQ, stg, hh * C::DH + wq * 32, i * C::BM + 32 * c, b * p.Hq + h);
+          bulk_commit();
+        }
+      }
     }
+    if (lane == 0) bulk_wait_all();  // the reduce-adds complete before exit
   }
 
   tc_fence_before();

@@ -187,15 +187,16 @@ fa_status bwd_launch(const void* q, const void* k, const void* v, const void* o,
     // one CTA per (128-key tile, batch * kv head, half of the head dimension); 64-row query
     // steps (bwd_d256.cuh)
     using C = Bwd256Cfg;
-    CUtensorMap mq, mk, mv, mo;
+    CUtensorMap mq, mk, mv, mo, mdq;
     if (!make_map_bf16(&mq, q, d, Nq, B * Hq, C::BM) || !make_map_bf16(&mk, k, d, Nkv, B * Hkv, C::BN) ||
-        !make_map_bf16(&mv, v, d, Nkv, B * Hkv, C::BN) || !make_map_bf16(&mo, dO, d, Nq, B * Hq, C::BM))
+        !make_map_bf16(&mv, v, d, Nkv, B * Hkv, C::BN) || !make_map_bf16(&mo, dO, d, Nq, B * Hq, C::BM) ||
+        !make_map_f32(&mdq, dq_acc, d, Nq, B * Hq))
       return FA_ERR_CUDA;
     BwdParams prm{dq_acc, lse2, dstat, dk, dv, grad_dtype == FA_DTYPE_BF16 ? 1 : 0, d, Hq, Hkv, Nq, Nkv, Nq_pad,
                   scale, scale * 1.4426950408889634f, g_wait_ns};
     auto kern = causal ? fa_bwd_d256_kernel<true> : fa_bwd_d256_kernel<false>;
     if (set_smem(kern, C::SMEM) != cudaSuccess) return FA_ERR_CUDA;
-    kern<<<dim3((Nkv + C::BN - 1) / C::BN, B * Hkv, 2), C::THREADS, C::SMEM, st>>>(mq, mk, mv, mo, prm);
+    kern<<<dim3((Nkv + C::BN - 1) / C::BN, B * Hkv, 2), C::THREADS, C::SMEM, st>>>(mq, mk, mv, mo, mdq, prm);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
     if (grad_dtype == FA_DTYPE_BF16) {
       const long n = long(rows) * d;
