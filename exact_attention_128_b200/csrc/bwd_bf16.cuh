@@ -224,8 +224,9 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
   volatile int* abort_flag = &bars->abort_flag;
 
   const int warp = warp_id(), lane = lane_id();
-  const int j = blockIdx.x;  // key tile (low j = most causal work: scheduled first)
-  const int bk = blockIdx.y;
+  const int nj = (p.Nkv + C::BN - 1) / C::BN;
+  int j, bk;  // key tile, (batch, kv head)
+  bwd_tile_order(blockIdx.x, nj, gridDim.x / nj, j, bk);
   const int b = bk / p.Hkv, hk = bk % p.Hkv;
   const int G = p.Hq / p.Hkv;
   const int off = p.Nkv - p.Nq;

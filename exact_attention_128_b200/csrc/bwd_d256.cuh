@@ -76,9 +76,11 @@ __global__ void __launch_bounds__(Bwd256Cfg::THREADS, 1)
   volatile int* abort_flag = &bars->abort_flag;
 
   const int warp = warp_id(), lane = lane_id();
-  const int j = blockIdx.x;  // key tile
-  const int bk = blockIdx.y;
-  const int hh = blockIdx.z;  // head-dimension half
+  const int nj = (p.Nkv + C::BN - 1) / C::BN;
+  int j, u;  // key tile, unit = (batch, kv head) x 2 + head-dimension half
+  bwd_tile_order(blockIdx.x, nj, gridDim.x / nj, j, u);
+  const int bk = u >> 1;
+  const int hh = u & 1;  // head-dimension half
   const int b = bk / p.Hkv, hk = bk % p.Hkv;
   const int G = p.Hq / p.Hkv;
   const int off = p.Nkv - p.Nq;

@@ -337,6 +337,22 @@ __device__ __forceinline__ float ex2(float x) {
 }
 
 // max(a, b, c) in one instruction (sm_100 three-input max).
+// Work order of the backward grids.  CTA `lin` of a 1-D grid over nj key tiles x nu units
+// (a (batch, kv head), or a (batch, kv head, head-dimension half)) takes key tile j of unit
+// u.  Units are taken kBwdGroup at a time, and inside a group tile 0 of every unit comes
+// before tile 1, and so on.  Under a causal mask tile j has the most work at j = 0, so the
+// CTAs that start last are the shortest (longest first), while the few units that run
+// together still share their query-side rows in L2.
+constexpr int kBwdGroup = 16;
+__device__ __forceinline__ void bwd_tile_order(int lin, int nj, int nu, int& j, int& u) {
+  const int grp = lin / (nj * kBwdGroup);
+  const int u0 = grp * kBwdGroup;
+  const int gs = min(kBwdGroup, nu - u0);  // units in this (possibly last, smaller) group
+  const int r = lin - grp * nj * kBwdGroup;
+  j = r / gs;
+  u = u0 + r % gs;
+}
+
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));

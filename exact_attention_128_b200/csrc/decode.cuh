@@ -374,23 +374,48 @@ __global__ void __launch_bounds__(128) fa_paged_decode_combine_kernel(const Deco
   const int nsplit = ((ctx + BS - 1) / BS + p.chunk - 1) / p.chunk;
   if (nsplit <= 1) return;
   const float* pl = p.part_lse + size_t(rh) * p.max_splits;
+  const float* po = p.part_o + size_t(rh) * p.max_splits * D;
+  const int d = threadIdx.x;
+  // The first NPRE splits' lse and output column are all loaded before any arithmetic that
+  // needs them, so their loads overlap (one L2 round trip instead of one per dependent
+  // step); splits past NPRE, if any, are read as they are merged.
+  constexpr int NPRE = 8;
+  float lv[NPRE], ov[NPRE];
+#pragma unroll
+  for (int s = 0; s < NPRE; ++s)
+    if (s < nsplit) {
+      lv[s] = pl[s];
+      ov[s] = po[size_t(s) * D + d];
+    }
   float M = -INFINITY;
   bool aborted = false;  // a split whose bounded wait ran out left NaN
-  for (int s = 0; s < nsplit; ++s) {
+#pragma unroll
+  for (int s = 0; s < NPRE; ++s)
+    if (s < nsplit) {
+      M = fmaxf(M, lv[s]);
+      aborted |= isnan(lv[s]);
+    }
+  for (int s = NPRE; s < nsplit; ++s) {
     M = fmaxf(M, pl[s]);
     aborted |= isnan(pl[s]);
   }
   if (aborted) {
-    p.o[size_t(rh) * D + threadIdx.x] = __float2bfloat16_rn(NAN);
-    if (threadIdx.x == 0 && p.lse) p.lse[rh] = NAN;
+    p.o[size_t(rh) * D + d] = __float2bfloat16_rn(NAN);
+    if (d == 0 && p.lse) p.lse[rh] = NAN;
     return;
   }
   float W = 0.f, U = 0.f;
-  const int d = threadIdx.x;
-  for (int s = 0; s < nsplit; ++s) {
+#pragma unroll
+  for (int s = 0; s < NPRE; ++s)
+    if (s < nsplit) {
+      const float w = __expf(lv[s] - M);
+      W += w;
+      U += w * ov[s];
+    }
+  for (int s = NPRE; s < nsplit; ++s) {
     const float w = __expf(pl[s] - M);
     W += w;
-    U += w * p.part_o[(size_t(rh) * p.max_splits + s) * D + d];
+    U += w * po[size_t(s) * D + d];
   }
   p.o[size_t(rh) * D + d] = __float2bfloat16_rn(U / W);
   if (d == 0 && p.lse) p.lse[rh] = M + __logf(W);

@@ -130,7 +130,8 @@ fa_status launch_bwd_kernel(const CUtensorMap& mq, const CUtensorMap& mk, const 
   using C = BwdCfg<D>;
   auto kern = fa_bwd_bf16_kernel<D, CAUSAL>;
   if (set_smem(kern, C::SMEM) != cudaSuccess) return FA_ERR_CUDA;
-  dim3 grid((Nkv + C::BN - 1) / C::BN, B * Hkv);
+  // 1-D grid over (key tile, (batch, kv head)) in the order bwd_tile_order gives
+  dim3 grid(((Nkv + C::BN - 1) / C::BN) * B * Hkv);
   kern<<<grid, C::THREADS, C::SMEM, st>>>(mq, mk, mv, mo, mdq, mdk, mdv, prm);
   return launched();
 }
@@ -196,7 +197,8 @@ fa_status bwd_launch(const void* q, const void* k, const void* v, const void* o,
                   scale, scale * 1.4426950408889634f, g_wait_ns};
     auto kern = causal ? fa_bwd_d256_kernel<true> : fa_bwd_d256_kernel<false>;
     if (set_smem(kern, C::SMEM) != cudaSuccess) return FA_ERR_CUDA;
-    kern<<<dim3((Nkv + C::BN - 1) / C::BN, B * Hkv, 2), C::THREADS, C::SMEM, st>>>(mq, mk, mv, mo, mdq, prm);
+    // 1-D grid over (key tile, (batch, kv head, half)) in the order bwd_tile_order gives
+    kern<<<dim3(((Nkv + C::BN - 1) / C::BN) * B * Hkv * 2), C::THREADS, C::SMEM, st>>>(mq, mk, mv, mo, mdq, prm);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
     if (grad_dtype == FA_DTYPE_BF16) {
       const long n = long(rows) * d;
