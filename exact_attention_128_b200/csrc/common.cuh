@@ -337,6 +337,14 @@ __device__ __forceinline__ float ex2(float x) {
 }
 
 // max(a, b, c) in one instruction (sm_100 three-input max).
+// k-th item of persistent CTA `cta` of `ncta`, in boustrophedon order: rounds of ncta
+// consecutive items, handed out forward in even rounds and backward in odd ones, so that
+// with items sorted longest first every CTA's total stays close to the mean (a plain
+// round-robin gives the low CTA indices the longest item of every round).
+__device__ __forceinline__ int snake_item(int k, int cta, int ncta) {
+  return k * ncta + ((k & 1) ? ncta - 1 - cta : cta);
+}
+
 // Work order of the backward grids.  CTA `lin` of a 1-D grid over nj key tiles x nu units
 // (a (batch, kv head), or a (batch, kv head, head-dimension half)) takes key tile j of unit
 // u.  Units are taken kBwdGroup at a time, and inside a group tile 0 of every unit comes

@@ -147,9 +147,12 @@ __global__ void __launch_bounds__(FwdCfg<D, BN>::THREADS, FwdCfg<D, BN>::CTAS_PE
   constexpr bool PAIRS = CAUSAL && !PAGED;
   const int n_units = (n_qp + 1) / 2;
   const int n_items = PAIRS ? 2 * n_units * p.BH : n_qp * p.BH;
-  // index of this CTA's k-th item (>= n_items once it has none left)
+  // index of this CTA's k-th item (>= n_items once it has none left): paired units and
+  // the equal non-causal items round-robin, the unequal paged causal items boustrophedon
   auto item_index = [&](int k) {
-    return PAIRS ? 2 * (int(blockIdx.x) + (k >> 1) * int(gridDim.x)) + (k & 1) : int(blockIdx.x) + k * int(gridDim.x);
+    if constexpr (PAIRS) return 2 * (int(blockIdx.x) + (k >> 1) * int(gridDim.x)) + (k & 1);
+    else if constexpr (CAUSAL) return snake_item(k, int(blockIdx.x), int(gridDim.x));
+    else return int(blockIdx.x) + k * int(gridDim.x);
   };
   // keys (L) and query rows (ql) of a sequence; paged mode reads them per request and
   // gives out-of-range lengths no work (flagging them in the status word)

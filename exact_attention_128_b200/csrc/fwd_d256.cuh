@@ -72,6 +72,11 @@ __global__ void __launch_bounds__(D256Cfg::THREADS, 1)
   const int off = p.Nkv - p.Nq;  // bottom-right causal alignment
   auto item_qt = [&](int it) { return CAUSAL ? n_qt - 1 - it / p.BH : it % n_qt; };
   auto item_bh = [&](int it) { return CAUSAL ? it % p.BH : it / n_qt; };
+  // this CTA's k-th item: boustrophedon order over the longest-first causal items,
+  // round-robin over the equal non-causal ones
+  auto item_at = [&](int k) {
+    return CAUSAL ? snake_item(k, int(blockIdx.x), int(gridDim.x)) : int(blockIdx.x) + k * int(gridDim.x);
+  };
   auto item_ntiles = [&](int qt) {
     const int kv_end = CAUSAL ? min(p.Nkv, min(qt * C::BM + C::BM, p.Nq) + off) : p.Nkv;
     return (kv_end + C::BN - 1) / C::BN;
@@ -110,7 +115,7 @@ __global__ void __launch_bounds__(D256Cfg::THREADS, 1)
       prefetch_tmap(&tmV);
       int kv = 0, local = 0;
       bool ok = true;
-      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++local) {
+      for (int k = 0, it = item_at(0); it < n_items && ok; it = item_at(++k), ++local) {
         const int qt = item_qt(it), bh = item_bh(it), n = item_ntiles(qt);
         const int zkv = (bh / p.Hq) * p.Hkv + (bh % p.Hq) / (p.Hq / p.Hkv);
         if (local > 0 && !(ok = mbar_wait(&bars->q_empty, (local - 1) & 1, p.wait_ns, abort_flag, 211))) break;
@@ -151,7 +156,7 @@ __global__ void __launch_bounds__(D256Cfg::THREADS, 1)
       };
       int kv = 0, g = 0, local = 0;
       bool ok = true;
-      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++local) {
+      for (int k = 0, it = item_at(0); it < n_items && ok; it = item_at(++k), ++local) {
         const int n = item_ntiles(item_qt(it));
         ok = mbar_wait(&bars->q_full, local & 1, p.wait_ns, abort_flag, 220) &&
              mbar_wait(&bars->k_full[kv & 1], (kv >> 1) & 1, p.wait_ns, abort_flag, 221);
@@ -193,7 +198,7 @@ __global__ void __launch_bounds__(D256Cfg::THREADS, 1)
     const float2 sl2v = make_float2(sl2, sl2);
     int g = 0, local = 0;
     bool ok = true;
-    for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++local) {
+    for (int k = 0, it = item_at(0); it < n_items && ok; it = item_at(++k), ++local) {
       const int qt = item_qt(it), bh = item_bh(it), n = item_ntiles(qt);
       const int row = qt * C::BM + r;
       const int row_limit = CAUSAL ? min(p.Nkv, row + off + 1) : p.Nkv;
