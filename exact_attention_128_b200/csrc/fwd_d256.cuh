@@ -46,7 +46,9 @@ struct D256Cfg {
 
 struct D256Bars {
   uint64_t q_full, q_empty;
-  uint64_t k_full[2], v_full[2], kv_empty[2];
+  uint64_t k_full[2], v_full[2];
+  uint64_t k_empty[2];  // the S that read a K stage has completed
+  uint64_t v_empty[2];  // the P.V that read a V stage has completed
   uint64_t s_full[2];  // per S buffer
   uint64_t p_full;     // P of the current tile written (4 softmax warps)
   uint64_t o_ready;    // the P.V of a tile has completed (one completion per tile)
@@ -88,7 +90,8 @@ __global__ void __launch_bounds__(D256Cfg::THREADS, 1)
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars->k_full[s], 1);
       mbar_init(&bars->v_full[s], 1);
-      mbar_init(&bars->kv_empty[s], 1);
+      mbar_init(&bars->k_empty[s], 1);
+      mbar_init(&bars->v_empty[s], 1);
       mbar_init(&bars->s_full[s], 1);
     }
     mbar_init(&bars->p_full, 4);
@@ -123,13 +126,18 @@ __global__ void __launch_bounds__(D256Cfg::THREADS, 1)
         for (int kb = 0; kb < C::KB; ++kb)
           tma_load_3d(smem + C::OFF_Q + kb * C::BM * 128, &tmQ, &bars->q_full, kb * 64, qt * C::BM, bh);
         for (int j = 0; j < n; ++j, ++kv) {
+          // K and V stages are released separately: a K stage as soon as the S that read it
+          // has run.  S of tile j + 2 is issued right after the P.V of tile j, so a K stage
+          // freed only by that P.V (as the V stage is) would make every S wait for its load.
           const int st = kv & 1, round = kv >> 1;
-          if (round > 0 && !(ok = mbar_wait(&bars->kv_empty[st], (round - 1) & 1, p.wait_ns, abort_flag, 210)))
+          if (round > 0 && !(ok = mbar_wait(&bars->k_empty[st], (round - 1) & 1, p.wait_ns, abort_flag, 210)))
             break;
           mbar_arrive_expect_tx(&bars->k_full[st], C::KV_TILE);
           for (int kb = 0; kb < C::KB; ++kb)
             tma_load_3d(smem + C::OFF_K + st * C::KV_TILE + kb * C::BN * 128, &tmK, &bars->k_full[st], kb * 64,
                         j * C::BN, zkv);
+          if (round > 0 && !(ok = mbar_wait(&bars->v_empty[st], (round - 1) & 1, p.wait_ns, abort_flag, 213)))
+            break;
           mbar_arrive_expect_tx(&bars->v_full[st], C::KV_TILE);
           for (int kb = 0; kb < C::KB; ++kb)
             tma_load_3d(smem + C::OFF_V + st * C::KV_TILE + kb * C::BN * 128, &tmV, &bars->v_full[st], kb * 64,
@@ -153,6 +161,7 @@ __global__ void __launch_bounds__(D256Cfg::THREADS, 1)
                  sdesc_sw128(sK + st * C::KV_TILE + kb * C::BN * 128 + kin * 32, 16, 1024), idS, ks > 0 ? 1u : 0u);
         }
         mma_commit(&bars->s_full[g & 1]);
+        mma_commit(&bars->k_empty[st]);
       };
       int kv = 0, g = 0, local = 0;
       bool ok = true;
@@ -182,7 +191,7 @@ __global__ void __launch_bounds__(D256Cfg::THREADS, 1)
             mma_ts(tmem + C::COL_O, tmem + C::COL_S + (g & 1) * C::BN + ks * 8,
                    sdesc_sw128(sV + st * C::KV_TILE + ks * 16 * 128, C::BN * 128, 1024), idPV,
                    (j > 0 || ks > 0) ? 1u : 0u);
-          mma_commit(&bars->kv_empty[st]);
+          mma_commit(&bars->v_empty[st]);
           mma_commit(&bars->o_ready);
           if (j + 1 == n) mma_commit(&bars->o_final);
         }
