@@ -53,7 +53,8 @@ struct Bwd256Bars {
   uint64_t v_tmem;  // V copied into TMEM (8 softmax-gradient warps arrive)
   uint64_t qdo_full[2];
   uint64_t qdo_empty[2];
-  uint64_t sdp_full;
+  uint64_t s_full;   // S^T of the step is in TMEM
+  uint64_t dp_full;  // dP^T of the step is in TMEM
   uint64_t ds_ready;
   uint64_t dq_full;
   uint64_t dq_free;
@@ -97,7 +98,8 @@ __global__ void __launch_bounds__(Bwd256Cfg::THREADS, 1)
       mbar_init(&bars->qdo_full[s], 1);
       mbar_init(&bars->qdo_empty[s], 1);
     }
-    mbar_init(&bars->sdp_full, 1);
+    mbar_init(&bars->s_full, 1);
+    mbar_init(&bars->dp_full, 1);
     mbar_init(&bars->ds_ready, 8);
     mbar_init(&bars->dq_full, 1);
     mbar_init(&bars->dq_free, 4);
@@ -166,6 +168,7 @@ __global__ void __launch_bounds__(Bwd256Cfg::THREADS, 1)
         for (int ks = 0; ks < 16; ++ks)
           mma_ss_p(tmem + C::COL_S, desc_add(dK, (ks >> 2) * 16384 + (ks & 3) * 32),
                    desc_add(dQk, qo + (ks >> 2) * 8192 + (ks & 3) * 32), idS, ks > 0, leader);
+        mma_commit_p(&bars->s_full, leader);
       };
       // dP^T = V dO^T with V from TMEM (8 columns = 16 bf16 per k-step)
       auto issue_dp = [&](int s) {
@@ -174,7 +177,7 @@ __global__ void __launch_bounds__(Bwd256Cfg::THREADS, 1)
         for (int ks = 0; ks < 16; ++ks)
           mma_ts_p(tmem + C::COL_DP, tmem + C::COL_VA + ks * 8, desc_add(dOk, qo + (ks >> 2) * 8192 + (ks & 3) * 32),
                    idS, ks > 0, leader);
-        mma_commit_p(&bars->sdp_full, leader);
+        mma_commit_p(&bars->dp_full, leader);
       };
       // dV_h += P^T dO[:, h] and dK_h += dS^T Q[:, h] (K dimension = 64 queries: 4 k-steps;
       // P^T / dS^T of queries 16k..16k+15 at columns (k >> 1) * 32 + (k & 1) * 8)
@@ -209,13 +212,16 @@ __global__ void __launch_bounds__(Bwd256Cfg::THREADS, 1)
         if (!(ok = warp_wait(&bars->ds_ready, s & 1, p.wait_ns, abort_flag, 313))) break;
         tc_fence_after();
         issue_dvdk(s);
-        // S^T of the next step may overwrite P^T now (the MMAs run in issue order)
+        // dQ^T of this step next (it reads dS^T from shared memory and writes over dS^T in
+        // TMEM after dK has read it: the MMAs run in issue order), so that its drain runs
+        // while S^T of the next step is computed
+        issue_dq();
+        // S^T of the next step may overwrite P^T now
         if (s + 1 < n_steps) {
           if (!(ok = warp_wait(&bars->qdo_full[(s + 1) & 1], ((s + 1) >> 1) & 1, p.wait_ns, abort_flag, 314))) break;
           tc_fence_after();
           issue_s(s + 1);
         }
-        issue_dq();
         if (s + 1 < n_steps) {
           // dP^T of the next step overwrites dQ^T: wait for its drain
           if (!(ok = warp_wait(&bars->dq_free, s & 1, p.wait_ns, abort_flag, 315))) break;
@@ -264,8 +270,10 @@ __global__ void __launch_bounds__(Bwd256Cfg::THREADS, 1)
     for (int s = 0; s < n_steps && ok; ++s) {
       const int st = s & 1;
       const int i = i_begin + s % n_i;
+      // P first, as soon as S^T has landed (the tensor core is meanwhile computing dP^T),
+      // then dS once dP^T has
       ok = warp_wait(&bars->qdo_full[st], (s >> 1) & 1, p.wait_ns, abort_flag, 321) &&
-           warp_wait(&bars->sdp_full, s & 1, p.wait_ns, abort_flag, 322);
+           warp_wait(&bars->s_full, s & 1, p.wait_ns, abort_flag, 322);
       if (!ok) break;
       tc_fence_after();
       int lim = 0;  // columns q < lim of this warp's 32 are masked for this key
@@ -275,17 +283,16 @@ __global__ void __launch_bounds__(Bwd256Cfg::THREADS, 1)
       const float* d_s = lse_s + 64;
       const bool any_masked = __any_sync(0xffffffffu, lim > 0);
       uint8_t* dsrow = smem + C::OFF_DS + r * 128;
+      float pr[32];  // P of this key and the warp's 32 queries
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
-        uint32_t sv[16], dv[16];
+        uint32_t sv[16];
         tmem_ld16(tmem + lane_off + C::COL_S + q0 + 16 * c, sv);
-        tmem_ld16(tmem + lane_off + C::COL_DP + q0 + 16 * c, dv);
         tmem_wait_ld();
-        uint32_t pp[8], pd[8];
+        uint32_t pp[8];
 #pragma unroll
         for (int e = 0; e < 16; e += 4) {
           const float4 l4 = *reinterpret_cast<const float4*>(lse_s + 16 * c + e);
-          const float4 d4 = *reinterpret_cast<const float4*>(d_s + 16 * c + e);
           const float2 x01 = __ffma2_rn(make_float2(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])),
                                         make_float2(sl2, sl2), make_float2(-l4.x, -l4.y));
           const float2 x23 = __ffma2_rn(make_float2(__uint_as_float(sv[e + 2]), __uint_as_float(sv[e + 3])),
@@ -299,20 +306,40 @@ __global__ void __launch_bounds__(Bwd256Cfg::THREADS, 1)
             if (col + 2 < lim) p23.x = 0.f;
             if (col + 3 < lim) p23.y = 0.f;
           }
-          // dS * scale = P * (dP * scale - D * scale)  (d4 holds D * scale)
-          const float2 g01 = __fmul2_rn(
-              p01, __ffma2_rn(make_float2(__uint_as_float(dv[e]), __uint_as_float(dv[e + 1])),
-                              make_float2(scale, scale), make_float2(-d4.x, -d4.y)));
-          const float2 g23 = __fmul2_rn(
-              p23, __ffma2_rn(make_float2(__uint_as_float(dv[e + 2]), __uint_as_float(dv[e + 3])),
-                              make_float2(scale, scale), make_float2(-d4.z, -d4.w)));
+          pr[16 * c + e] = p01.x;
+          pr[16 * c + e + 1] = p01.y;
+          pr[16 * c + e + 2] = p23.x;
+          pr[16 * c + e + 3] = p23.y;
           pp[e / 2] = pack_bf16x2(p01.x, p01.y);
           pp[e / 2 + 1] = pack_bf16x2(p23.x, p23.y);
+        }
+        // packed P^T of queries 16k..16k+15 at columns (k >> 1) * 32 + (k & 1) * 8
+        tmem_st8(tmem + lane_off + C::COL_S + q0 + 8 * c, pp);
+      }
+      if (!(ok = warp_wait(&bars->dp_full, s & 1, p.wait_ns, abort_flag, 324))) break;
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t dv[16];
+        tmem_ld16(tmem + lane_off + C::COL_DP + q0 + 16 * c, dv);
+        tmem_wait_ld();
+        uint32_t pd[8];
+#pragma unroll
+        for (int e = 0; e < 16; e += 4) {
+          const float4 d4 = *reinterpret_cast<const float4*>(d_s + 16 * c + e);
+          // dS * scale = P * (dP * scale - D * scale)  (d4 holds D * scale)
+          const float2 g01 = __fmul2_rn(
+              make_float2(pr[16 * c + e], pr[16 * c + e + 1]),
+              __ffma2_rn(make_float2(__uint_as_float(dv[e]), __uint_as_float(dv[e + 1])), make_float2(scale, scale),
+                         make_float2(-d4.x, -d4.y)));
+          const float2 g23 = __fmul2_rn(
+              make_float2(pr[16 * c + e + 2], pr[16 * c + e + 3]),
+              __ffma2_rn(make_float2(__uint_as_float(dv[e + 2]), __uint_as_float(dv[e + 3])), make_float2(scale, scale),
+                         make_float2(-d4.z, -d4.w)));
           pd[e / 2] = pack_bf16x2(g01.x, g01.y);
           pd[e / 2 + 1] = pack_bf16x2(g23.x, g23.y);
         }
-        // packed P^T / dS^T of queries 16k..16k+15 at columns (k >> 1) * 32 + (k & 1) * 8
-        tmem_st8(tmem + lane_off + C::COL_S + q0 + 8 * c, pp);
+        // packed dS^T at the same columns, over dP^T
         tmem_st8(tmem + lane_off + C::COL_DP + q0 + 8 * c, pd);
         // dS^T row r: [64 queries] of 128 bytes, 16-byte unit q/8 at unit ^ (r % 8)
 #pragma unroll
