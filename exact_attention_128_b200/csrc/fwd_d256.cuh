@@ -10,7 +10,8 @@
 // holds ONE query tile (not the d <= 128 kernel's two).  The tensor core is kept busy by
 // double-buffering the score tile instead: S for key tile j+1 is computed into one
 // 64-column buffer while the softmax works on tile j in the other.
-// TMEM: S/P buffers at columns [0, 64) and [64, 128), O at [256, 512).
+// TMEM: S/P buffers at columns [0, 64) and [64, 128), Q at [128, 256) (bf16 pairs, the A
+// operand of S = Q K^T, so that S reads only K from shared memory), O at [256, 512).
 // Shared memory: Q (64 KB, four 64-column blocks), two K/V stages of 64 keys (32 KB each
 // for K and V), per-warp epilogue staging.
 //   warp 0      TMA producer (one thread)
@@ -41,11 +42,14 @@ struct D256Cfg {
   static constexpr int THREADS = 256;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t COL_S = 0;  // + (tile & 1) * BN
+  static constexpr uint32_t COL_QA = 128;
   static constexpr uint32_t COL_O = 256;
 };
 
 struct D256Bars {
-  uint64_t q_full, q_empty;
+  uint64_t q_full, q_empty;  // Q in shared memory loaded / copied out (4 softmax warps arrive)
+  uint64_t q_tmem;           // Q copied into TMEM (4 softmax warps arrive)
+  uint64_t q_tmem_free;      // the item's last S, the last reader of Q in TMEM, has run
   uint64_t k_full[2], v_full[2];
   uint64_t k_empty[2];  // the S that read a K stage has completed
   uint64_t v_empty[2];  // the P.V that read a V stage has completed
@@ -86,7 +90,9 @@ __global__ void __launch_bounds__(D256Cfg::THREADS, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
-    mbar_init(&bars->q_empty, 1);
+    mbar_init(&bars->q_empty, 4);
+    mbar_init(&bars->q_tmem, 4);
+    mbar_init(&bars->q_tmem_free, 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars->k_full[s], 1);
       mbar_init(&bars->v_full[s], 1);
@@ -150,14 +156,14 @@ __global__ void __launch_bounds__(D256Cfg::THREADS, 1)
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16_f32(128, C::BN, 0);  // K-major Q and K
       constexpr uint32_t idPV = idesc_bf16_f32(128, C::D, 1);  // V is MN-major
-      const uint32_t sQ = smem_u32(smem + C::OFF_Q), sK = smem_u32(smem + C::OFF_K);
+      const uint32_t sK = smem_u32(smem + C::OFF_K);
       const uint32_t sV = smem_u32(smem + C::OFF_V);
       // S of key tile g (global tile count) into buffer g & 1
       auto issue_S = [&](int st, int g) {
 #pragma unroll
         for (int ks = 0; ks < C::D / 16; ++ks) {
           const int kb = ks >> 2, kin = ks & 3;
-          mma_ss(tmem + C::COL_S + (g & 1) * C::BN, sdesc_sw128(sQ + kb * C::BM * 128 + kin * 32, 16, 1024),
+          mma_ts(tmem + C::COL_S + (g & 1) * C::BN, tmem + C::COL_QA + ks * 8,
                  sdesc_sw128(sK + st * C::KV_TILE + kb * C::BN * 128 + kin * 32, 16, 1024), idS, ks > 0 ? 1u : 0u);
         }
         mma_commit(&bars->s_full[g & 1]);
@@ -167,12 +173,12 @@ __global__ void __launch_bounds__(D256Cfg::THREADS, 1)
       bool ok = true;
       for (int k = 0, it = item_at(0); it < n_items && ok; it = item_at(++k), ++local) {
         const int n = item_ntiles(item_qt(it));
-        ok = mbar_wait(&bars->q_full, local & 1, p.wait_ns, abort_flag, 220) &&
+        ok = mbar_wait(&bars->q_tmem, local & 1, p.wait_ns, abort_flag, 220) &&
              mbar_wait(&bars->k_full[kv & 1], (kv >> 1) & 1, p.wait_ns, abort_flag, 221);
         if (!ok) break;
         tc_fence_after();
         issue_S(kv & 1, g);
-        if (n == 1) mma_commit(&bars->q_empty);
+        if (n == 1) mma_commit(&bars->q_tmem_free);
         for (int j = 0; j < n; ++j, ++kv, ++g) {
           const int st = kv & 1;
           if (j + 1 < n) {
@@ -180,7 +186,7 @@ __global__ void __launch_bounds__(D256Cfg::THREADS, 1)
             if (!(ok = mbar_wait(&bars->k_full[st ^ 1], ((kv + 1) >> 1) & 1, p.wait_ns, abort_flag, 222))) break;
             tc_fence_after();
             issue_S(st ^ 1, g + 1);
-            if (j + 2 == n) mma_commit(&bars->q_empty);  // the item's last S
+            if (j + 2 == n) mma_commit(&bars->q_tmem_free);  // the item's last S
           }
           ok = mbar_wait(&bars->v_full[st], (kv >> 1) & 1, p.wait_ns, abort_flag, 223) &&
                mbar_wait(&bars->p_full, g & 1, p.wait_ns, abort_flag, 224);
@@ -205,8 +211,39 @@ __global__ void __launch_bounds__(D256Cfg::THREADS, 1)
     const uint32_t tO = tmem + lane_off + C::COL_O;
     const float sl2 = p.scale_log2;
     const float2 sl2v = make_float2(sl2, sl2);
+    // Q of the CTA's item number `lq` from shared memory into TMEM: row r (TMEM lane r) as
+    // 128 columns of bf16 pairs in d order, the A-operand layout of the TS MMA.  Every warp
+    // copies its 32 rows, idle or not.  Item lq's copy waits for item lq - 1's last S.
+    auto copy_q = [&](int lq) -> bool {
+      if (lq > 0 && !warp_wait(&bars->q_tmem_free, (lq - 1) & 1, p.wait_ns, abort_flag, 234)) return false;
+      if (!warp_wait(&bars->q_full, lq & 1, p.wait_ns, abort_flag, 235)) return false;
+      tc_fence_after();
+#pragma unroll 1
+      for (int kb = 0; kb < C::KB; ++kb) {
+        const uint8_t* qrow = smem + C::OFF_Q + kb * C::BM * 128 + r * 128;  // 128-byte swizzle
+        uint32_t a[32];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const uint4 x = *reinterpret_cast<const uint4*>(qrow + ((u ^ (r & 7)) << 4));
+          a[4 * u] = x.x;
+          a[4 * u + 1] = x.y;
+          a[4 * u + 2] = x.z;
+          a[4 * u + 3] = x.w;
+        }
+        tmem_st32(tmem + lane_off + C::COL_QA + kb * 32, a);
+      }
+      tmem_wait_st();
+      fence_proxy_async_smem();  // these reads precede the TMA writes of the next Q
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&bars->q_tmem);
+        mbar_arrive(&bars->q_empty);
+      }
+      return true;
+    };
     int g = 0, local = 0;
-    bool ok = true;
+    bool ok = item_at(0) < n_items ? copy_q(0) : true;
     for (int k = 0, it = item_at(0); it < n_items && ok; it = item_at(++k), ++local) {
       const int qt = item_qt(it), bh = item_bh(it), n = item_ntiles(qt);
       const int row = qt * C::BM + r;
@@ -288,6 +325,9 @@ __global__ void __launch_bounds__(D256Cfg::THREADS, 1)
         if (lane == 0) mbar_arrive(&bars->p_full);
       }
       if (!ok) break;
+      // the next item's Q goes into TMEM now (this item's last S has run), so its first S
+      // overlaps this item's epilogue
+      if (item_at(k + 1) < n_items && !(ok = copy_q(local + 1))) break;
       if (!(ok = warp_wait(&bars->o_final, local & 1, p.wait_ns, abort_flag, 232))) break;
       if (idle) continue;
       tc_fence_after();
