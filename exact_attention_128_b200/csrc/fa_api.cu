@@ -317,9 +317,9 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   if (d != 64 && d != 96 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
 
   if (d == 256) {  // one query tile per CTA, double-buffered scores (fwd_d256.cuh)
-    CUtensorMap mq, mk, mv, mo;
+    CUtensorMap mq, mk, mv;
     if (!make_map_bf16(&mq, q, d, Nq, B * Hq, D256Cfg::BM) || !make_map_bf16(&mk, k, d, Nkv, B * Hkv, D256Cfg::BN) ||
-        !make_map_bf16(&mv, v, d, Nkv, B * Hkv, D256Cfg::BN) || !make_map_bf16(&mo, o, d, Nq, B * Hq, 32))
+        !make_map_bf16(&mv, v, d, Nkv, B * Hkv, D256Cfg::BN))
       return FA_ERR_CUDA;
     FwdBf16Params prm{static_cast<__nv_bfloat16*>(o), lse, B * Hq, Hq, Hkv, Nq, Nkv,
                       scale * 1.4426950408889634f, g_wait_ns, nullptr, nullptr, nullptr, 0, 0};
@@ -328,7 +328,7 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
     const long items = long((Nq + D256Cfg::BM - 1) / D256Cfg::BM) * B * Hq;
     const long slots = sm_count();
     if (slots <= 0) return FA_ERR_CUDA;
-    kern<<<int(items < slots ? items : slots), D256Cfg::THREADS, D256Cfg::SMEM, st>>>(mq, mk, mv, mo, prm);
+    kern<<<int(items < slots ? items : slots), D256Cfg::THREADS, D256Cfg::SMEM, st>>>(mq, mk, mv, prm);
     return launched();
   }
   constexpr int BN64 = FA_FWD_D64_BN;  // key-tile width of the d = 64 kernel
