@@ -303,6 +303,13 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
     if (d != 64) return FA_ERR_UNSUPPORTED;
     FwdF32Params prm{static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
                      static_cast<float*>(o), lse, Hq, Hkv, Nq, Nkv, scale, causal};
+    if (Nkv <= f32::SMALL_NKV) {
+      // every key of a head fits in shared memory: one pass per 32-row CTA
+      const size_t sb = fwd_f32_small_smem(Nkv);
+      if (set_smem(fa_fwd_f32_small_kernel, int(sb)) != cudaSuccess) return FA_ERR_CUDA;
+      fa_fwd_f32_small_kernel<<<dim3((Nq + f32::SROWS - 1) / f32::SROWS, B * Hq), f32::STHREADS, sb, st>>>(prm);
+      return launched();
+    }
     // 64-row CTAs, or 16-row CTAs when the former would leave SMs idle (a single ViT layer
     // has 4 x 12 of them for 148 SMs)
     if (long((Nq + 63) / 64) * B * Hq < 2L * sm_count()) {
