@@ -347,7 +347,8 @@ def measure_dense_fwd(case, dev, steps, warmup, world, peaks, peak_key="bf16_tfl
     tflops = flops / sec / 1e12
     gbs = nbytes / sec / 1e9
     if case.dtype == "f32":
-        kname = "fa_fwd_f32_kernel"
+        # up to 256 keys the library runs its one-pass fp32 kernel, above that the tiled one
+        kname = "fa_fwd_f32_small_kernel" if case.Nkv <= 256 else "fa_fwd_f32_kernel"
         peak = fp32_alu_peak_tflops(peaks)
         roof = {"bound": "alu", "achieved": round(tflops, 3), "peak": round(peak, 1), "unit": "TFLOP/s",
                 "frac": round(tflops / peak, 4), "peak_kind": "fp32 FFMA, 148 SMs x 128 lanes x 2 x max clock",
