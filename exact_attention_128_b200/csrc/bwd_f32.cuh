@@ -60,12 +60,23 @@ __global__ void __launch_bounds__(256) fa_bwd_f32_pre_kernel(const float* o, con
 
 namespace b32 {
 
-// rows [r0, r0 + BR) of a [n, 64] matrix into a padded tile; rows past n read as zero
+// rows [r0, r0 + BR) of a [n, 64] matrix into a padded tile; rows past n read as zero.
+// Each of the 8 * BR threads loads its D / 8 elements before storing any, so the loads'
+// latencies overlap instead of adding up.
 template <int BR>
 __device__ __forceinline__ void load_tile(float (*dst)[RP], const float* src, int r0, int n) {
-  for (int e = threadIdx.x; e < BR * D; e += 8 * BR) {
+  constexpr int PER = D / 8;
+  float x[PER];
+#pragma unroll
+  for (int u = 0; u < PER; ++u) {
+    const int e = threadIdx.x + u * 8 * BR;
     const int r = e / D, c = e % D;
-    dst[r][c] = (r0 + r < n) ? src[size_t(r0 + r) * D + c] : 0.f;
+    x[u] = (r0 + r < n) ? src[size_t(r0 + r) * D + c] : 0.f;
+  }
+#pragma unroll
+  for (int u = 0; u < PER; ++u) {
+    const int e = threadIdx.x + u * 8 * BR;
+    dst[e / D][e % D] = x[u];
   }
 }
 

@@ -81,17 +81,31 @@ __global__ void __launch_bounds__(4 * BQ) fa_fwd_f32_kernel(const FwdF32Params p
 
   for (int t = 0; t < ntiles; ++t) {
     const int k0 = t * BK;
-    // stage K (padded rows) and V tiles; rows past Nkv are zero
-    for (int i = tid; i < BK * (D / 4); i += THREADS) {
-      const int kr = i / (D / 4), c4 = (i % (D / 4)) * 4;
-      float4 kk = make_float4(0, 0, 0, 0), vv = make_float4(0, 0, 0, 0);
-      if (k0 + kr < p.Nkv) {
-        kk = *reinterpret_cast<const float4*>(Kh + size_t(k0 + kr) * D + c4);
-        vv = *reinterpret_cast<const float4*>(Vh + size_t(k0 + kr) * D + c4);
+    // stage K (padded rows) and V tiles; rows past Nkv are zero.  A thread's loads are all
+    // issued before its first store, so their latencies overlap.
+    {
+      constexpr int IT = BK * (D / 4) / THREADS;
+      static_assert(IT * THREADS == BK * (D / 4), "the tile splits evenly over the threads");
+      float4 kk[IT], vv[IT];
+#pragma unroll
+      for (int u = 0; u < IT; ++u) {
+        const int i = tid + u * THREADS;
+        const int kr = i / (D / 4), c4 = (i % (D / 4)) * 4;
+        kk[u] = make_float4(0, 0, 0, 0);
+        vv[u] = make_float4(0, 0, 0, 0);
+        if (k0 + kr < p.Nkv) {
+          kk[u] = *reinterpret_cast<const float4*>(Kh + size_t(k0 + kr) * D + c4);
+          vv[u] = *reinterpret_cast<const float4*>(Vh + size_t(k0 + kr) * D + c4);
+        }
       }
-      float* kd = Ks + kr * KPAD + c4;
-      kd[0] = kk.x; kd[1] = kk.y; kd[2] = kk.z; kd[3] = kk.w;
-      *reinterpret_cast<float4*>(Vs + kr * D + c4) = vv;
+#pragma unroll
+      for (int u = 0; u < IT; ++u) {
+        const int i = tid + u * THREADS;
+        const int kr = i / (D / 4), c4 = (i % (D / 4)) * 4;
+        float* kd = Ks + kr * KPAD + c4;
+        kd[0] = kk[u].x; kd[1] = kk[u].y; kd[2] = kk[u].z; kd[3] = kk[u].w;
+        *reinterpret_cast<float4*>(Vs + kr * D + c4) = vv[u];
+      }
     }
     __syncthreads();
 
