@@ -10,13 +10,15 @@
 // (the gradient of sum(O * dO) by matrix calculus; dK and dV summed over the query heads
 // that share a key/value head).
 //
-// fp32 inputs need fp32 products, so this path uses FFMA, like the fp32 forward.  Three
+// fp32 inputs need fp32 products, so this path uses FFMA, like the fp32 forward.  Two
 // kernels, no atomics, every result written once:
 //   fa_bwd_f32_pre_kernel   D_i, one warp per query row
-//   fa_bwd_f32_dkdv_kernel  one CTA per (BR-key block, batch, kv head): walks the group's
-//                           query heads and the query blocks that see the keys
-//   fa_bwd_f32_dq_kernel    one CTA per (BR-row query block, batch, query head): walks
-//                           the key blocks the rows see
+//   fa_bwd_f32_kernel       two kinds of CTA in one grid, which run side by side (each kind
+//                           alone leaves the SMs with few warps to hide its latencies):
+//     dK/dV CTA  one per (BR-key block, batch, kv head): walks the group's query heads and
+//                the query blocks that see the keys
+//     dQ CTA     one per (BR-row query block, batch, query head): walks the key blocks the
+//                rows see
 // Each step recomputes a BR x BR score tile in shared memory (8 threads per row, BR/8
 // scores each) and accumulates 8 output columns per thread; the library launches BR = 32.
 #pragma once
@@ -119,12 +121,24 @@ __device__ __forceinline__ void p_ds_tile(const float (*sQ)[RP], const float (*s
 }  // namespace b32
 
 template <int BR>
-__global__ void __launch_bounds__(8 * BR) fa_bwd_f32_dkdv_kernel(const BwdF32Params p) {
+struct BwdF32Smem {
+  float sK[BR][b32::RP], sV[BR][b32::RP], sQ[BR][b32::RP], sdO[BR][b32::RP];
+  float sP[BR][BR + 1], sS[BR][BR + 1], sL[BR], sD[BR];
+};
+
+// dK and dV of key block kb of (batch, kv head) bk
+template <int BR>
+__device__ __forceinline__ void bwd_f32_dkdv(const BwdF32Params& p, BwdF32Smem<BR>& sm, int kb, int bk) {
   using namespace b32;
   constexpr int BQ = BR, BK = BR;
-  __shared__ float sK[BK][RP], sV[BK][RP], sQ[BQ][RP], sdO[BQ][RP];
-  __shared__ float sP[BQ][BR + 1], sS[BQ][BR + 1], sL[BQ], sD[BQ];
-  const int kb = blockIdx.x, bk = blockIdx.y;  // key block; batch * Hkv + kv head
+  auto& sK = sm.sK;
+  auto& sV = sm.sV;
+  auto& sQ = sm.sQ;
+  auto& sdO = sm.sdO;
+  auto& sP = sm.sP;
+  auto& sS = sm.sS;
+  auto& sL = sm.sL;
+  auto& sD = sm.sD;
   const int b = bk / p.Hkv, hk = bk % p.Hkv, G = p.Hq / p.Hkv;
   const int kj0 = kb * BK;
   load_tile<BR>(sK, p.k + size_t(bk) * p.Nkv * D, kj0, p.Nkv);
@@ -175,13 +189,19 @@ __global__ void __launch_bounds__(8 * BR) fa_bwd_f32_dkdv_kernel(const BwdF32Par
   }
 }
 
+// dQ of query block qb of (batch, query head) bh
 template <int BR>
-__global__ void __launch_bounds__(8 * BR) fa_bwd_f32_dq_kernel(const BwdF32Params p) {
+__device__ __forceinline__ void bwd_f32_dq(const BwdF32Params& p, BwdF32Smem<BR>& sm, int qb, int bh) {
   using namespace b32;
   constexpr int BQ = BR, BK = BR;
-  __shared__ float sK[BK][RP], sV[BK][RP], sQ[BQ][RP], sdO[BQ][RP];
-  __shared__ float sP[BQ][BR + 1], sS[BQ][BR + 1], sL[BQ], sD[BQ];
-  const int qb = blockIdx.x, bh = blockIdx.y;  // query block; batch * Hq + head
+  auto& sK = sm.sK;
+  auto& sV = sm.sV;
+  auto& sQ = sm.sQ;
+  auto& sdO = sm.sdO;
+  auto& sP = sm.sP;
+  auto& sS = sm.sS;
+  auto& sL = sm.sL;
+  auto& sD = sm.sD;
   const int b = bh / p.Hq, h = bh % p.Hq;
   const size_t bk = size_t(b) * p.Hkv + h / (p.Hq / p.Hkv);
   const int qi0 = qb * BQ;
@@ -219,6 +239,18 @@ __global__ void __launch_bounds__(8 * BR) fa_bwd_f32_dq_kernel(const BwdF32Param
 #pragma unroll
     for (int u = 0; u < 8; ++u) dq[u] = adq[u] * p.scale;
   }
+}
+
+// CTAs [0, n_dkdv) compute dK/dV (key block, batch * Hkv + kv head), the rest dQ (query
+// block, batch * Hq + query head); both index orders are key/query block fastest.
+template <int BR>
+__global__ void __launch_bounds__(8 * BR) fa_bwd_f32_kernel(const BwdF32Params p, int n_kb, int n_dkdv, int n_qb) {
+  __shared__ BwdF32Smem<BR> sm;
+  const int c = blockIdx.x;
+  if (c < n_dkdv)
+    bwd_f32_dkdv<BR>(p, sm, c % n_kb, c / n_kb);
+  else
+    bwd_f32_dq<BR>(p, sm, (c - n_dkdv) % n_qb, (c - n_dkdv) / n_qb);
 }
 
 }  // namespace fa

@@ -428,8 +428,13 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
     fa_bwd_f32_pre_kernel<<<unsigned((rows + 7) / 8), 256, 0, st>>>(prm.o, prm.dO, prm.Dvec, rows);
     // 32-row blocks (16-row blocks, though they fill more SMs on a single ViT layer, were
     // measured slower: 197 vs 185 us for that layer's forward + backward)
-    fa_bwd_f32_dkdv_kernel<32><<<dim3((Nkv + 31) / 32, B * Hkv), 256, 0, st>>>(prm);
-    fa_bwd_f32_dq_kernel<32><<<dim3((Nq + 31) / 32, B * Hq), 256, 0, st>>>(prm);
+    {
+      // the dK/dV and the dQ CTAs in one grid, so that they share the SMs
+      const long n_kb = (Nkv + 31) / 32, n_qb = (Nq + 31) / 32;
+      const long n_dkdv = n_kb * B * Hkv, n_all = n_dkdv + n_qb * B * Hq;
+      if (n_all > 0x7fffffffL) return FA_ERR_UNSUPPORTED;
+      fa_bwd_f32_kernel<32><<<unsigned(n_all), 256, 0, st>>>(prm, int(n_kb), int(n_dkdv), int(n_qb));
+    }
     return launched();
   }
   if (dtype != FA_DTYPE_BF16) return FA_ERR_UNSUPPORTED;
