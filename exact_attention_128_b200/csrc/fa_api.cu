@@ -118,7 +118,19 @@ fa_status launch_fwd_bf16(const CUtensorMap& mq, const CUtensorMap& mk, const CU
   const long items = (CAUSAL && !PAGED ? (n_qp + 1) / 2 : n_qp) * prm.BH;
   const long slots = long(sm_count()) * C::CTAS_PER_SM;
   if (slots <= 0) return FA_ERR_CUDA;
-  kern<<<int(items < slots ? items : slots), C::THREADS, C::SMEM, st>>>(mq, mk, mv, mo, prm);
+  // programmatic dependent launch (the kernel waits for the preceding grid before any
+  // global access): its launch and prologue overlap the tail of the kernel before it
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned(items < slots ? items : slots));
+  cfg.blockDim = dim3(C::THREADS);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, mo, prm) != cudaSuccess) return FA_ERR_CUDA;
   return launched();
 }
 

@@ -231,6 +231,13 @@ __global__ void __launch_bounds__(FwdCfg<D, BN>::THREADS, FwdCfg<D, BN>::CTAS_PE
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // Launched as a programmatic dependent: everything above touches only this CTA's shared
+  // memory and TMEM, so its launch and set-up overlap the tail of the grid before it.  Wait
+  // here, before any global access, until that grid has completed and its writes are
+  // visible.  (No early trigger for the grid after this one: with it the causal d = 64
+  // forward ran 20 % slower, its CTAs finishing at different times; each CTA's exit triggers
+  // it instead.)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const uint32_t tmem = bars->tmem_base;
   const uint32_t sQ = smem_u32(smem + C::OFF_Q);
   const uint32_t sK = smem_u32(smem + C::OFF_K);
