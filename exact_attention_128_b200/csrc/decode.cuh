@@ -97,6 +97,10 @@ __global__ void __launch_bounds__(dec::WARPS * 32)
   uint8_t* dsmem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) & ~uintptr_t(1023));
   const int s = blockIdx.x, g = blockIdx.y, r = blockIdx.z;
   const int G = p.Hq / p.Hkv;
+  // launched as a programmatic dependent: wait for the grid before it on the stream (the
+  // previous step's merge, or the append that wrote this step's key/value rows) to
+  // complete before reading anything it may have written; the launch itself overlaps it
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int ctx = p.ctx[r];
   if (ctx < 1 || ctx > p.max_blocks * BS) {
     if (s == 0 && g == 0 && threadIdx.x == 0) set_status(FA_ERR_INVALID_ARG, 100);

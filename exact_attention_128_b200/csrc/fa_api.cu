@@ -518,8 +518,21 @@ fa_status fa_paged_decode(const void* q, const void* k_cache, const void* v_cach
   if (!make_map_cache(&mk, k_cache, cache_rows) || !make_map_cache(&mv, v_cache, cache_rows)) return FA_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (set_smem(fa_paged_decode_kernel, dec::SMEM) != cudaSuccess) return FA_ERR_CUDA;
-  fa_paged_decode_kernel<<<dim3(max_splits, Hkv, R), dec::WARPS * 32, dec::SMEM, st>>>(mk, mv, prm);
-  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  {
+    // programmatic dependent launch: the split kernel waits (griddepcontrol.wait) for the
+    // grid before it, so its launch overlaps that grid's tail
+    cudaLaunchConfig_t c = {};
+    c.gridDim = dim3(max_splits, Hkv, R);
+    c.blockDim = dim3(dec::WARPS * 32);
+    c.dynamicSmemBytes = dec::SMEM;
+    c.stream = st;
+    cudaLaunchAttribute a[1];
+    a[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    a[0].val.programmaticStreamSerializationAllowed = 1;
+    c.attrs = a;
+    c.numAttrs = 1;
+    if (cudaLaunchKernelEx(&c, fa_paged_decode_kernel, mk, mv, prm) != cudaSuccess) return FA_ERR_CUDA;
+  }
   // the merge is a programmatic dependent launch: its launch overlaps the split kernel's
   // tail and it waits (griddepcontrol.wait) for the split kernel's results
   cudaLaunchConfig_t cfg = {};
