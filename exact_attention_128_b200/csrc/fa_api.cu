@@ -4,6 +4,7 @@
 #include <cmath>
 #include <cstdio>
 #include <mutex>
+#include <utility>
 
 #include "common.cuh"
 #include "decode.cuh"
@@ -99,6 +100,26 @@ cudaError_t set_smem(K kernel, int bytes) {
 
 fa_status launched() { return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA; }
 
+// Launch `kernel` as a programmatic dependent on stream st: it may be launched while the
+// grid before it is still finishing.  Every kernel launched this way executes
+// griddepcontrol.wait before its first global access, which returns once that grid has
+// completed and its writes are visible.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args&&... args) {
+  cudaLaunchConfig_t c = {};
+  c.gridDim = grid;
+  c.blockDim = block;
+  c.dynamicSmemBytes = smem;
+  c.stream = st;
+  cudaLaunchAttribute a[1];
+  a[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  a[0].val.programmaticStreamSerializationAllowed = 1;
+  c.attrs = a;
+  c.numAttrs = 1;
+  return cudaLaunchKernelEx(&c, kernel, std::forward<Args>(args)...);
+}
+
 // Number of SMs of the current device (persistent grids use one CTA per SM).
 int sm_count() {
   int dev = 0, n = 0;
@@ -118,19 +139,10 @@ fa_status launch_fwd_bf16(const CUtensorMap& mq, const CUtensorMap& mk, const CU
   const long items = (CAUSAL && !PAGED ? (n_qp + 1) / 2 : n_qp) * prm.BH;
   const long slots = long(sm_count()) * C::CTAS_PER_SM;
   if (slots <= 0) return FA_ERR_CUDA;
-  // programmatic dependent launch (the kernel waits for the preceding grid before any
-  // global access): its launch and prologue overlap the tail of the kernel before it
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(unsigned(items < slots ? items : slots));
-  cfg.blockDim = dim3(C::THREADS);
-  cfg.dynamicSmemBytes = C::SMEM;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, mo, prm) != cudaSuccess) return FA_ERR_CUDA;
+  // programmatic dependent: its launch and prologue overlap the tail of the grid before it
+  if (launch_pdl(kern, dim3(unsigned(items < slots ? items : slots)), dim3(C::THREADS), C::SMEM, st, mq, mk, mv, mo,
+                 prm) != cudaSuccess)
+    return FA_ERR_CUDA;
   return launched();
 }
 
@@ -518,21 +530,10 @@ fa_status fa_paged_decode(const void* q, const void* k_cache, const void* v_cach
   if (!make_map_cache(&mk, k_cache, cache_rows) || !make_map_cache(&mv, v_cache, cache_rows)) return FA_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (set_smem(fa_paged_decode_kernel, dec::SMEM) != cudaSuccess) return FA_ERR_CUDA;
-  {
-    // programmatic dependent launch: the split kernel waits (griddepcontrol.wait) for the
-    // grid before it, so its launch overlaps that grid's tail
-    cudaLaunchConfig_t c = {};
-    c.gridDim = dim3(max_splits, Hkv, R);
-    c.blockDim = dim3(dec::WARPS * 32);
-    c.dynamicSmemBytes = dec::SMEM;
-    c.stream = st;
-    cudaLaunchAttribute a[1];
-    a[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    a[0].val.programmaticStreamSerializationAllowed = 1;
-    c.attrs = a;
-    c.numAttrs = 1;
-    if (cudaLaunchKernelEx(&c, fa_paged_decode_kernel, mk, mv, prm) != cudaSuccess) return FA_ERR_CUDA;
-  }
+  // programmatic dependent: the split kernel's launch overlaps the tail of the grid before it
+  if (launch_pdl(fa_paged_decode_kernel, dim3(max_splits, Hkv, R), dim3(dec::WARPS * 32), dec::SMEM, st, mk, mv,
+                 prm) != cudaSuccess)
+    return FA_ERR_CUDA;
   // the merge is a programmatic dependent launch: its launch overlaps the split kernel's
   // tail and it waits (griddepcontrol.wait) for the split kernel's results
   cudaLaunchConfig_t cfg = {};
