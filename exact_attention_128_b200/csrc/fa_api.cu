@@ -1,6 +1,7 @@
 // fa_api.cu — the C ABI (include/fa.h): argument validation, TMA descriptor
 // encoding and kernel launches.  Everything that computes runs in the kernels;
 // this file only checks arguments and launches them on the caller's stream.
+#include <algorithm>
 #include <cmath>
 #include <cstdio>
 #include <mutex>
@@ -407,9 +408,13 @@ fa_status fa_paged_prefill(const void* q, const void* k_cache, const void* v_cac
   if (!make_map_bf16(&mq, q, d, Nq_max, R * Hq, 128) || !make_map_bf16(&mo, o, d, Nq_max, R * Hq, 32, stg_cols) ||
       !make_map_cache(&mk, k_cache, cache_rows, d) || !make_map_cache(&mv, v_cache, cache_rows, d))
     return FA_ERR_CUDA;
+  // causal item order: requests in groups whose K/V (bounded by the block table's width)
+  // takes at most 32 MB, a quarter of L2, so that it stays there while the group runs
+  const long kv_bytes = long(Hkv) * max_blocks_per_seq * 16 * d * 2 * 2;
+  const int group = int(std::max(1L, std::min(long(R), (32L << 20) / kv_bytes)));
   FwdBf16Params prm{static_cast<__nv_bfloat16*>(o), lse, R * Hq, Hq, Hkv, Nq_max, 0,
                     scale * 1.4426950408889634f, g_wait_ns, block_table, ctx_lens, q_lens, max_blocks_per_seq,
-                    num_blocks};
+                    num_blocks, group};
   if (d == 64)
     return causal ? launch_fwd_bf16<64, BN64, true, true>(mq, mk, mv, mo, prm, Nq_max, st)
                   : launch_fwd_bf16<64, BN64, false, true>(mq, mk, mv, mo, prm, Nq_max, st);

@@ -11,8 +11,9 @@
 // Persistent kernel: CTAs walk work items (two 128-row query tiles Q0, Q1 of one (batch,
 // query head)), item = blockIdx.x + k * gridDim.x, ordered head-major (non-causal: K/V
 // reuse in L2); causal items go in head-major units of a long and a short item of equal
-// total length (paged causal: longest-first).  Each item streams the 128-key tiles of its key/value head (GQA: head
-// h reads h / (Hq/Hkv)).  The K/V ring and the Q buffers run ahead across item
+// total length (paged causal: requests in L2-sized groups, longest first inside a group).
+// Each item streams the 128-key tiles of its key/value head (GQA: head h reads
+// h / (Hq/Hkv)).  The K/V ring and the Q buffers run ahead across item
 // boundaries, so loads for the next item overlap the current item's tail and epilogue.
 //   warp 0      TMA producer: Q0/Q1 per item (QBUF buffers), K_j and V_j into a ring.
 //   warp 1      MMA issuer (the warp runs the role, one elected lane issues): S_t = Q_t K_j^T
@@ -79,6 +80,10 @@ struct FwdCfg {
   static constexpr int OFF_V = OFF_K + NSTAGE * KV_TILE;
   static constexpr int OFF_STG = OFF_V + NSTAGE * KV_TILE;  // epilogue staging, per softmax warp
   static constexpr int OFF_BAR = OFF_STG + 8 * STG_WARP;
+  // paged causal prefill: the requests' order, longest first (PERM_MAX requests at most)
+  static constexpr int PERM_MAX = 256;
+  static constexpr int OFF_PERM = OFF_BAR + 256;
+  static constexpr int END = OFF_PERM + 4 * PERM_MAX;
   static constexpr int WG0 = (BN == 64) ? 2 : 4;     // first softmax warp
   static constexpr int THREADS = 32 * (WG0 + 8);
   static constexpr int CTAS_PER_SM = (BN == 64) ? 2 : 1;
@@ -86,10 +91,11 @@ struct FwdCfg {
   // when that is what lets CTAS_PER_SM blocks share the SM's 228 KB (1 KB of it reserved
   // per block); the kernel checks at run time that the slack it needs is there
   static constexpr int SMEM_CAP = 233472 / CTAS_PER_SM - 1024;
-  static constexpr int SLACK = (SMEM_CAP - (OFF_BAR + 256)) < 1024 ? (SMEM_CAP - (OFF_BAR + 256)) : 1024;
+  static constexpr int SLACK = (SMEM_CAP - END) < 1024 ? (SMEM_CAP - END) : 1024;
   static_assert(SLACK >= 0, "shared memory over budget");
   static_assert(NSTAGE <= 4, "barrier arrays hold 4 stages");
-  static constexpr int SMEM = OFF_BAR + 256 + SLACK;  // + barriers + alignment slack
+  static_assert(8 * STG_WARP >= 4 * PERM_MAX, "the request lengths are sorted in the staging area");
+  static constexpr int SMEM = END + SLACK;  // + barriers, request order, alignment slack
   static constexpr uint32_t TMEM_COLS = (BN == 64) ? 256 : 512;
   static constexpr uint32_t COL_S = 0;       // + t * BN
   static constexpr uint32_t COL_O = 2 * BN;  // + t * D
@@ -106,6 +112,7 @@ struct FwdBf16Params {
   const int* ctx;   // cached tokens of request b (the keys)
   const int* qlen;  // query rows of request b (the last qlen positions of its sequence)
   int max_blocks, num_blocks;
+  int group;  // paged causal: requests per group of the item order (>= 1)
 };
 
 struct FwdBars {
@@ -147,13 +154,15 @@ __global__ void __launch_bounds__(FwdCfg<D, BN>::THREADS, FwdCfg<D, BN>::CTAS_PE
   constexpr bool PAIRS = CAUSAL && !PAGED;
   const int n_units = (n_qp + 1) / 2;
   const int n_items = PAIRS ? 2 * n_units * p.BH : n_qp * p.BH;
-  // index of this CTA's k-th item (>= n_items once it has none left): paired units and
-  // the equal non-causal items round-robin, the unequal paged causal items boustrophedon
+  // index of this CTA's k-th item (>= n_items once it has none left), round-robin; paired
+  // units go to one CTA whole
   auto item_index = [&](int k) {
     if constexpr (PAIRS) return 2 * (int(blockIdx.x) + (k >> 1) * int(gridDim.x)) + (k & 1);
-    else if constexpr (CAUSAL) return snake_item(k, int(blockIdx.x), int(gridDim.x));
     else return int(blockIdx.x) + k * int(gridDim.x);
   };
+  // paged causal: the requests by query rows, longest first (filled after the grid
+  // dependency wait below; with more than PERM_MAX requests the request order is kept)
+  const int* s_perm = reinterpret_cast<const int*>(smem + C::OFF_PERM);
   // keys (L) and query rows (ql) of a sequence; paged mode reads them per request and
   // gives out-of-range lengths no work (flagging them in the status word)
   auto seq_len = [&](int bh, int& L, int& ql) {
@@ -175,8 +184,11 @@ __global__ void __launch_bounds__(FwdCfg<D, BN>::THREADS, FwdCfg<D, BN>::CTAS_PE
   // nothing to do).  Non-causal items are head-major, so the CTAs running at the same time
   // share one or two heads' K/V in L2 (at N = 8192 this cut DRAM traffic per launch from
   // 4.2 GB to the 0.64 GB of the algorithm); causal items are the paired units above.  In
-  // paged mode the causal order is longest-first over all heads, counting tile pairs from
-  // each request's own last one, so the long items of every request come first.
+  // paged mode the causal items go by groups of p.group requests (the host sizes a group
+  // so that its K/V stays in L2 while every query tile of the group reads it), the groups
+  // and the requests inside them longest first; inside a group, rank k of the tile pairs
+  // counted from each request's own last one, then the request, then the head: so the
+  // long items of a group run first and its short ones fill the gaps at its end.
   struct Item {
     int qt, bh, L, ql, n;
   };
@@ -189,13 +201,19 @@ __global__ void __launch_bounds__(FwdCfg<D, BN>::THREADS, FwdCfg<D, BN>::CTAS_PE
       seq_len(x.bh, x.L, x.ql);
       x.qt = (it & 1) ? a : n_qp - 1 - a;
       if ((it & 1) && x.qt == n_qp - 1 - a) return x;  // the unpaired middle pair
-    } else {
-      x.bh = CAUSAL ? it % p.BH : it / n_qp;
+    } else if constexpr (CAUSAL) {  // paged (dense causal items are the paired units)
+      const int n_req = p.BH / p.Hq, per_req = n_qp * p.Hq;  // item slots of one request
+      const int g = it / (p.group * per_req), g_n = min(p.group, n_req - g * p.group);
+      const int in_g = it - g * p.group * per_req;
+      const int rank = in_g / (g_n * p.Hq);
+      const int j = in_g - rank * g_n * p.Hq, pos = g * p.group + j / p.Hq;
+      x.bh = (n_req <= C::PERM_MAX ? s_perm[pos] : pos) * p.Hq + j % p.Hq;
       seq_len(x.bh, x.L, x.ql);
-      if (CAUSAL && PAGED)
-        x.qt = (x.ql + 2 * C::BM - 1) / (2 * C::BM) - 1 - it / p.BH;
-      else
-        x.qt = CAUSAL ? n_qp - 1 - it / p.BH : it % n_qp;
+      x.qt = (x.ql + 2 * C::BM - 1) / (2 * C::BM) - 1 - rank;
+    } else {
+      x.bh = it / n_qp;
+      seq_len(x.bh, x.L, x.ql);
+      x.qt = it % n_qp;
     }
     if (x.qt >= 0 && x.qt * 2 * C::BM < x.ql) {
       int kv_end = x.L;
@@ -238,6 +256,25 @@ __global__ void __launch_bounds__(FwdCfg<D, BN>::THREADS, FwdCfg<D, BN>::CTAS_PE
   // forward ran 20 % slower, its CTAs finishing at different times; each CTA's exit triggers
   // it instead.)
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  if constexpr (CAUSAL && PAGED) {
+    // rank each request by its query rows (descending, ties by index: a strict order, so
+    // the ranks are a permutation) against a copy of the lengths in the epilogue staging
+    // area, which no epilogue has used yet
+    const int n_req = p.BH / p.Hq;
+    if (n_req <= C::PERM_MAX) {
+      int* s_len = reinterpret_cast<int*>(smem + C::OFF_STG);
+      int* perm = reinterpret_cast<int*>(smem + C::OFF_PERM);
+      for (int r = threadIdx.x; r < n_req; r += blockDim.x) s_len[r] = __ldg(p.qlen + r);
+      __syncthreads();
+      for (int r = threadIdx.x; r < n_req; r += blockDim.x) {
+        const int key = s_len[r];
+        int pos = 0;
+        for (int t = 0; t < n_req; ++t) pos += (s_len[t] > key) || (s_len[t] == key && t < r);
+        perm[pos] = r;
+      }
+    }
+    __syncthreads();
+  }
   const uint32_t tmem = bars->tmem_base;
   const uint32_t sQ = smem_u32(smem + C::OFF_Q);
   const uint32_t sK = smem_u32(smem + C::OFF_K);

@@ -61,6 +61,39 @@ def test_paged_prefill_vs_oracle(d, Hq, Hkv, ctx, ql, causal):
     check_rows(o, lse, O, L, inp["q_lens"], f"d={d}")
 
 
+@pytest.mark.parametrize(
+    "d,Hq,Hkv,width,ctx,ql",
+    [
+        # the causal item order takes requests in groups whose K/V, bounded by the block
+        # table's width, fits 32 MB: Hkv 2 x 8192 blocks at d = 128 makes groups of one,
+        (128, 4, 2, 8192, (300, 1000, 17, 1000, 513), None),
+        # 1 x 1536 blocks at d = 128 groups of two (the last one partial), with equal lengths
+        (128, 4, 1, 1536, (700, 129, 700, 256, 1), (700, 129, 45, 256, 1)),
+        # 2 x 1024 blocks at d = 64 groups of four (the last one partial)
+        (64, 4, 2, 1024, (300, 65, 777, 300, 20, 512, 513), (300, 65, 1, 129, 20, 512, 257)),
+    ],
+)
+def test_paged_prefill_causal_request_groups(d, Hq, Hkv, width, ctx, ql):
+    """Wide block tables make the causal prefill run its requests in several groups (sorted
+    by length inside the kernel): the result matches the oracle and equals, bit for bit,
+    the run over the same table cut to the blocks in use (one group), since every item
+    computes the same tiles in the same order whatever item order the CTAs follow."""
+    pc = PagedPrefillCase("groups", len(ctx), Hq, Hkv, d, 16, 1, 8192, width, True, 80 + Hq + d,
+                          ctx_lens_override=ctx, q_lens_override=ql)
+    inp = pc.make(poison=True)
+    fa.device_status(reset=True)
+    o, lse = run(inp, True)
+    assert fa.device_status() == 0
+    O, L = oracle(inp, True)
+    check_rows(o, lse, O, L, inp["q_lens"], f"width={width}")
+    narrow = dict(inp, block_table=inp["block_table"][:, :(max(ctx) + 15) // 16].contiguous())
+    o1, lse1 = run(narrow, True)
+    assert fa.device_status() == 0
+    for r, n in enumerate(inp["q_lens"].tolist()):
+        assert torch.equal(o[r, :, :n], o1[r, :, :n]), f"request {r}"
+        assert torch.equal(lse[r, :, :n], lse1[r, :, :n]), f"request {r}"
+
+
 def test_paged_prefill_matches_dense_kernel_bitwise():
     """Whole causal prompts over the paged cache give exactly the dense forward's bits on
     the same (de-paged) keys and values: the tiles and their order are the same."""
