@@ -443,6 +443,34 @@ def test_paged_prefill_equals_dense_and_decode():
         ora.paged_prefill(q, kc, vc, table, ctx, [2, 10, 3], bs, 0.5, True)
 
 
+def test_paged_prefill_chunk_equals_last_rows_of_whole_prompt():
+    """A prompt chunk (the last q_len < ctx positions of a sequence whose earlier part is
+    cached) gives exactly the last q_len rows of the whole prompt's result, causal or not:
+    each chunk row sees the cached prefix and the chunk up to its own position."""
+    rng = np.random.default_rng(23)
+    Hq, Hkv, d, bs = 4, 2, 3, 4
+    ctx, qlen = [5, 9, 13], [2, 4, 7]
+    R = len(ctx)
+    ks = [rng.standard_normal((Hkv, n, d)) for n in ctx]
+    vs = [rng.standard_normal((Hkv, n, d)) for n in ctx]
+    kc, table = _scatter_to_pages(ks, bs, Hkv, d, np.random.default_rng(5))
+    vc, _ = _scatter_to_pages(vs, bs, Hkv, d, np.random.default_rng(5))
+    qw = rng.standard_normal((R, Hq, max(ctx), d))
+    qc = np.zeros((R, Hq, max(qlen), d))
+    for r in range(R):
+        qc[r, :, :qlen[r]] = qw[r, :, ctx[r] - qlen[r]:ctx[r]]
+    for causal in (False, True):
+        Ow, Lw = ora.paged_prefill(qw, kc, vc, table, ctx, ctx, bs, 0.5, causal)
+        Oc, Lc = ora.paged_prefill(qc, kc, vc, table, ctx, qlen, bs, 0.5, causal)
+        for r in range(R):
+            np.testing.assert_allclose(Oc[r, :, :qlen[r]], Ow[r, :, ctx[r] - qlen[r]:ctx[r]], atol=1e-14)
+            np.testing.assert_allclose(Lc[r, :, :qlen[r]], Lw[r, :, ctx[r] - qlen[r]:ctx[r]], atol=1e-14)
+    # and the causal chunk is not the non-causal one (the mask reaches into the chunk)
+    Oc0, _ = ora.paged_prefill(qc, kc, vc, table, ctx, qlen, bs, 0.5, False)
+    Oc1, _ = ora.paged_prefill(qc, kc, vc, table, ctx, qlen, bs, 0.5, True)
+    assert not np.allclose(Oc0[2, :, :qlen[2] - 1], Oc1[2, :, :qlen[2] - 1])
+
+
 def test_single_key_gradients_are_zero_in_the_oracle():
     """With one key every softmax row is [1], so dS = P (dP - D) = 0 and dQ = dK = 0 up to
     fp64 rounding (the case the parity checker compares by max-abs only)."""
