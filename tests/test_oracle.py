@@ -255,6 +255,29 @@ def test_gradients_match_torch_fp64_autograd():
         np.testing.assert_allclose(dv, v.grad.numpy(), atol=1e-12)
 
 
+@pytest.mark.parametrize("Nq,Nkv,causal", [(3, 9, True), (7, 9, True), (3, 9, False), (9, 4, False)])
+def test_gradients_rectangular_match_torch_fp64_autograd(Nq, Nkv, causal):
+    """Nq != Nkv, with the causal mask aligned bottom-right (query i sees keys
+    j <= i + Nkv - Nq), given to torch as an explicit boolean mask."""
+    g = torch.Generator().manual_seed(16)
+    B, Hq, Hkv, d = 1, 4, 2, 5
+    q = torch.randn(B, Hq, Nq, d, generator=g, dtype=torch.float64, requires_grad=True)
+    k = torch.randn(B, Hkv, Nkv, d, generator=g, dtype=torch.float64, requires_grad=True)
+    v = torch.randn(B, Hkv, Nkv, d, generator=g, dtype=torch.float64, requires_grad=True)
+    do = torch.randn(B, Hq, Nq, d, generator=g, dtype=torch.float64)
+    mask = None
+    if causal:
+        mask = torch.arange(Nkv)[None, :] <= torch.arange(Nq)[:, None] + (Nkv - Nq)
+    out = torch.nn.functional.scaled_dot_product_attention(
+        q, k.repeat_interleave(2, 1), v.repeat_interleave(2, 1), attn_mask=mask, scale=0.4
+    )
+    out.backward(do)
+    dq, dk, dv = ora.attention_bwd(q.detach(), k.detach(), v.detach(), do, 0.4, causal)
+    np.testing.assert_allclose(dq, q.grad.numpy(), atol=1e-12)
+    np.testing.assert_allclose(dk, k.grad.numpy(), atol=1e-12)
+    np.testing.assert_allclose(dv, v.grad.numpy(), atol=1e-12)
+
+
 def test_gradient_invariants():
     """Softmax ignores a common shift of all keys, and P's rows sum to one."""
     rng = np.random.default_rng(14)
